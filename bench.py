@@ -1,0 +1,423 @@
+"""Benchmark: k-MIP attention query-heads/s, forward and forward+backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gmm_n100000] [--k 15]
+
+One step is the whole hot path over one batch: the forward (work list,
+fused score + top-k + softmax + V gather) and the backward (recompute,
+dQ, dK/dV scatter) of one graph of N = 100,000 nodes, 4 heads of 32, k = 15,
+keys from a 64-component Gaussian mixture.  The value is N * H / step time,
+summed over ranks.  With N > 1 GPUs (torchrun) every rank runs its own
+independent batch (a different seed) -- there is no data-path collective;
+the only collectives are the barriers and the max-over-ranks of the time.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; between steps a 256 MiB buffer is written to flush
+the L2 (126 MB), outside the events.  A barrier and a device synchronise
+bracket the whole timed loop.  One JSON line is printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from graph_transformer_sparse_kmip_b200 import binding  # noqa: E402
+from graph_transformer_sparse_kmip_b200 import workloads as wl  # noqa: E402
+
+METRIC = "k-MIP attn query-heads/s fwd & fwd+bwd at N=1e5; % of B200 bf16 tensor peak"
+UNIT = "query-heads/s"
+FWD_KERNEL_SOURCE = os.path.join(ROOT, "graph_transformer_sparse_kmip_b200", "csrc")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _score_flops(offsets: torch.Tensor, H: int, d: int) -> float:
+    n = torch.diff(offsets.long()).double()
+    return float(2.0 * d * H * (n * n).sum())
+
+
+def _kernel_hash(names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(FWD_KERNEL_SOURCE, n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else null)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(kernel_key)
+    except Exception:
+        return None
+    if not d or d.get("source_sha") != _kernel_hash(d.get("sources", [])):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        self.idx = str(device.index or 0)
+        try:  # nvidia-smi numbers GPUs physically; the UUID is unambiguous
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if uuid:
+                self.idx = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _flush(buf):
+    buf.add_(1)  # read + write 256 MiB: evicts the 126 MB L2
+
+
+def run_ours(args, ws, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    binding.load()
+    w = wl.WORKLOADS[args.workload]
+    k = args.k or w.k
+    inp = wl.make_inputs(w, with_grad_out=True, seed=w.seed + 7919 * rank)
+    N, H, d = inp["Q"].shape
+    scale = w.scale
+    g = {n: t.to(dev) for n, t in inp.items()}
+    stream = torch.cuda.current_stream()
+    out = torch.empty_like(g["Q"])
+    idx = torch.empty((N, H, k), dtype=torch.int32, device=dev)
+    lse = torch.empty((N, H), dtype=torch.float32, device=dev)
+    dQ = torch.empty((N, H, d), dtype=torch.float32, device=dev)
+    dK = torch.empty_like(dQ)
+    dV = torch.empty_like(dQ)
+    flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+
+    def step():
+        rc = binding.kmip_attn_fwd(g["Q"], g["K"], g["V"], g["offsets"], N, H, d, k, scale,
+                                   out, idx, lse, stream)
+        if rc:
+            raise binding.KmipError(rc, "kmip_attn_fwd")
+        ev_mid.record(stream)
+        rc = binding.kmip_attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, dQ, dK, dV,
+                                   stream, N, H, d, k, scale)
+        if rc:
+            raise binding.KmipError(rc, "kmip_attn_bwd")
+
+    ev_mid = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        step()
+        _flush(flush)
+    torch.cuda.synchronize()
+    binding.check_status()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        for s in range(args.steps):
+            a, m, b = evs[s]
+            a.record(stream)
+            ev_mid = m
+            step()
+            b.record(stream)
+            _flush(flush)
+        torch.cuda.synchronize()
+        if ws > 1:
+            torch.distributed.barrier()
+    binding.check_status()
+    fwd_ms = [a.elapsed_time(m) for a, m, _ in evs]
+    tot_ms = [a.elapsed_time(b) for a, _, b in evs]
+    t_fwd, t_tot = sum(fwd_ms), sum(tot_ms)
+    if ws > 1:
+        t = torch.tensor([t_fwd, t_tot], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_fwd, t_tot = t.tolist()
+    ms_step = t_tot / args.steps
+    ms_fwd = t_fwd / args.steps
+    units = N * H * ws
+    value = units / (ms_step * 1e-3)
+    fwd_value = units / (ms_fwd * 1e-3)
+
+    peaks, peak_kind = _peaks()
+    flops = _score_flops(inp["offsets"], H, d)
+    achieved = flops / (ms_fwd * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+
+    # k sweep (rank 0 view; fwd+bwd ms per step, same timing rules, fewer steps)
+    sweep = {}
+    if args.k_sweep and w.k_sweep:
+        for ks in w.k_sweep:
+            if ks == k:
+                sweep[str(ks)] = {"ms_fwd": round(ms_fwd, 4), "ms_fwd_bwd": round(ms_step, 4)}
+                continue
+            idx_s = torch.empty((N, H, ks), dtype=torch.int32, device=dev)
+            times = []
+            for it in range(args.warmup + max(3, args.steps // 2)):
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+                binding.kmip_attn_fwd(g["Q"], g["K"], g["V"], g["offsets"], N, H, d, ks, scale,
+                                      out, idx_s, lse, stream)
+                e1.record(stream)
+                binding.kmip_attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx_s, lse, dQ, dK, dV,
+                                      stream, N, H, d, ks, scale)
+                e2.record(stream)
+                _flush(flush)
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    times.append((e0.elapsed_time(e1), e0.elapsed_time(e2)))
+            sweep[str(ks)] = {"ms_fwd": round(statistics.mean(t[0] for t in times), 4),
+                              "ms_fwd_bwd": round(statistics.mean(t[1] for t in times), 4)}
+        binding.check_status()
+
+    # end to end through the public API: pinned host inputs in, host results out
+    e2e = None
+    if args.e2e:
+        hostin = {n: inp[n].pin_memory() for n in ("Q", "K", "V", "dO")}
+        off_h = inp["offsets"].pin_memory()
+        hostout = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                   "idx": torch.empty(idx.shape, dtype=idx.dtype).pin_memory(),
+                   "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory(),
+                   "dQ": torch.empty(dQ.shape, dtype=dQ.dtype).pin_memory(),
+                   "dK": torch.empty(dK.shape, dtype=dK.dtype).pin_memory(),
+                   "dV": torch.empty(dV.shape, dtype=dV.dtype).pin_memory()}
+        dbuf = {n: torch.empty_like(g[n]) for n in ("Q", "K", "V", "dO")}
+        doff = torch.empty_like(g["offsets"])
+        h2d = sum(t.numel() * t.element_size() for t in hostin.values()) + off_h.numel() * 4
+        d2h = sum(t.numel() * t.element_size() for t in hostout.values())
+
+        def e2e_step():
+            for n in dbuf:
+                dbuf[n].copy_(hostin[n], non_blocking=True)
+            doff.copy_(off_h, non_blocking=True)
+            binding.kmip_attn_fwd(dbuf["Q"], dbuf["K"], dbuf["V"], doff, N, H, d, k, scale,
+                                  out, idx, lse, stream)
+            binding.kmip_attn_bwd(dbuf["dO"], dbuf["Q"], dbuf["K"], dbuf["V"], idx, lse, dQ, dK,
+                                  dV, stream, N, H, d, k, scale)
+            for n, t in (("out", out), ("idx", idx), ("lse", lse), ("dQ", dQ), ("dK", dK),
+                         ("dV", dV)):
+                hostout[n].copy_(t, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if ws > 1:
+            torch.distributed.barrier()
+        e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e_b.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = e_a.elapsed_time(e_b)
+        if ws > 1:
+            t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            t_e2e = t.item()
+        binding.check_status()
+        e2e = {"value": units / (t_e2e / args.steps * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": t_e2e / args.steps}
+
+    cpu = None
+    if rank == 0 and ws == 1 and args.cpu_baseline:
+        cpu = cpu_baseline(inp, k, scale, budget_s=args.cpu_seconds)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "H": H, "d": d, "k": k, "graphs": int(
+            inp["offsets"].numel() - 1), "keys": w.values, "step": "fwd+bwd",
+            "parallelism": f"independent batch per GPU x{ws}",
+            "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "fwd": {"value": fwd_value, "unit": UNIT, "ms_per_step": ms_fwd},
+        "roofline": {"bound": "tensor", "kernel": "forward (score + top-k + softmax + gather)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": _traffic("fwd"),
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": flops},
+        "gpu_launches": 3 * args.steps,
+    }
+    if sweep:
+        res["k_sweep"] = sweep
+    if e2e:
+        res["e2e"] = e2e
+    if cpu:
+        res["cpu_baseline"] = cpu
+    res["clocks"] = clk.summary()
+    return res
+
+
+def cpu_baseline(inp, k, scale, budget_s=15.0, pairs_per_batch=None):
+    """The fp64 oracle, as it stands, on a bounded sample of (query, head)
+    pairs of the same workload: selection against all keys, softmax, V sum,
+    then the backward over the sampled pairs' sets.  Returns fwd+bwd
+    query-heads/s."""
+    import numpy as np
+
+    import oracle
+    N, H = inp["Q"].shape[:2]
+    threads = oracle.default_threads()
+    Qd = oracle._f64(inp["Q"]); Kd = oracle._f64(inp["K"]); Vd = oracle._f64(inp["V"])
+    dOd = oracle._f64(inp["dO"])
+    per = pairs_per_batch or max(64, threads * 8)
+    done, t_used, batch = 0, 0.0, 0
+    while t_used < budget_s and done < N * H:
+        pq, ph = wl.sample_pairs(N, H, per, seed=1000 + batch)
+        t0 = time.perf_counter()
+        r = oracle.fwd_pairs(Qd, Kd, Vd, inp["offsets"], k, scale, pq.numpy(), ph.numpy(),
+                             nthreads=threads)
+        full = np.full((N, H, k), -1, dtype=np.int32)
+        full[pq.numpy(), ph.numpy()] = r["idx"]
+        oracle.given_idx(Qd, Kd, Vd, full, inp["offsets"], scale, dO=dOd)
+        t_used += time.perf_counter() - t0
+        done += len(pq)
+        batch += 1
+    return {"value": done / t_used, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} (query, head) pairs of the same workload in {batch} batches; "
+                      f"fwd (all-key fp64 scores + full sort) and bwd; {t_used:.1f} s"}
+
+
+def run_reference(args, ws, rank):
+    """The oracle as the reference arm: bounded sample per step, host cores."""
+    if rank != 0:
+        return None
+    w = wl.WORKLOADS[args.workload]
+    k = args.k or w.k
+    inp = wl.make_inputs(w, with_grad_out=True)
+    N, H = inp["Q"].shape[:2]
+    per_step_s = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    vals, samples = [], []
+    for s in range(args.warmup + args.steps):
+        r = cpu_baseline(inp, k, w.scale, budget_s=per_step_s)
+        if s >= args.warmup:
+            vals.append(r["value"])
+            samples.append(r)
+    value = statistics.mean(vals)
+    ms_step = N * H / value * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "H": H, "d": w.d, "k": k, "step": "fwd+bwd",
+                   "parallelism": "host cores (oracle)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[-1]["cores"],
+                         "kind": "oracle", "sample": samples[-1]["sample"] + " per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gmm_n100000", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--no-k-sweep", dest="k_sweep", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws, rank, local = _dist()
+    if args.impl == "reference":
+        res = run_reference(args, ws, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

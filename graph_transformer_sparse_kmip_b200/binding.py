@@ -1,0 +1,152 @@
+"""Thin ctypes binding of libkmip (the C ABI declared in include/kmip.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libkmip.so.  torch provides device memory and streams.  There is
+no CPU fallback -- if the library is missing, or the tensors are not on a
+CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkmip.so")
+
+KMIP_BF16, KMIP_F32 = 0, 1
+STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTED",
+                3: "KMIP_ERR_CUDA", 4: "KMIP_ERR_BAD_OFFSETS", 5: "KMIP_ERR_TIMEOUT",
+                6: "KMIP_ERR_BAD_INDEX"}
+EXPORTED = ("kmip_attn_fwd", "kmip_attn_bwd", "kmip_get_status", "kmip_error_string",
+            "kmip_version")
+
+_lib = None
+
+
+class KmipError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}")
+
+
+def load() -> ctypes.CDLL:
+    """Load libkmip.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkmip.so not found at {LIB_PATH}; build it with "
+                          "`python -m graph_transformer_sparse_kmip_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, F32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    lib.kmip_attn_fwd.argtypes = [P, P, P, P, I64, I32, I32, I32, F32, P, P, P, P, I32, I32]
+    lib.kmip_attn_fwd.restype = I32
+    lib.kmip_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, F32, I32]
+    lib.kmip_attn_bwd.restype = I32
+    lib.kmip_get_status.argtypes = [P]
+    lib.kmip_get_status.restype = I32
+    lib.kmip_error_string.argtypes = [I32]
+    lib.kmip_error_string.restype = ctypes.c_char_p
+    lib.kmip_version.argtypes = []
+    lib.kmip_version.restype = I32
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return KMIP_BF16
+    if t == torch.float32:
+        return KMIP_F32
+    raise TypeError(f"unsupported dtype {t} (bf16 or fp32)")
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("libkmip takes contiguous CUDA tensors")
+
+
+# --- the C entry points, same names, torch tensors in place of pointers ---
+
+def kmip_attn_fwd(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, stream=None,
+                  num_graphs=None, dtype=None) -> int:
+    _check_cuda(Q, K, V, graph_offsets, out, idx, lse)
+    G = (graph_offsets.numel() - 1) if graph_offsets is not None else 1
+    if num_graphs is None:
+        num_graphs = G
+    if dtype is None:
+        dtype = dtype_code(Q.dtype)
+    return load().kmip_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N), int(H),
+                                int(d), int(k), float(scale), _ptr(out), _ptr(idx), _ptr(lse),
+                                _stream(stream), int(num_graphs), int(dtype))
+
+
+def kmip_attn_bwd(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None, N=None, H=None, d=None,
+                  k=None, scale=None, dtype=None) -> int:
+    _check_cuda(dOut, Q, K, V, idx, lse, dQ, dK, dV)
+    N_, H_, d_ = Q.shape
+    N = N_ if N is None else N
+    H = H_ if H is None else H
+    d = d_ if d is None else d
+    k = idx.shape[-1] if k is None else k
+    if dtype is None:
+        dtype = dtype_code(Q.dtype)
+    return load().kmip_attn_bwd(_ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse),
+                                _ptr(dQ), _ptr(dK), _ptr(dV), _stream(stream), int(N), int(H),
+                                int(d), int(k), float(scale), int(dtype))
+
+
+def kmip_get_status(stream=None) -> int:
+    return load().kmip_get_status(_stream(stream))
+
+
+def kmip_error_string(code: int) -> str:
+    return load().kmip_error_string(int(code)).decode()
+
+
+def kmip_version() -> int:
+    return load().kmip_version()
+
+
+# --- convenience wrappers that allocate the outputs with torch ---
+
+def attn_fwd(Q, K, V, k: int, scale: float, graph_offsets=None, stream=None):
+    """Returns (out [N,H,d] like Q, idx [N,H,k] int32, lse [N,H] fp32)."""
+    N, H, d = Q.shape
+    out = torch.empty_like(Q)
+    idx = torch.empty((N, H, k), dtype=torch.int32, device=Q.device)
+    lse = torch.empty((N, H), dtype=torch.float32, device=Q.device)
+    rc = kmip_attn_fwd(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, stream)
+    if rc:
+        raise KmipError(rc, "kmip_attn_fwd")
+    return out, idx, lse
+
+
+def attn_bwd(dOut, Q, K, V, idx, lse, scale: float, stream=None):
+    """Returns (dQ, dK, dV), fp32 [N,H,d]."""
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    dK = torch.empty_like(dQ)
+    dV = torch.empty_like(dQ)
+    rc = kmip_attn_bwd(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream, scale=scale)
+    if rc:
+        raise KmipError(rc, "kmip_attn_bwd")
+    return dQ, dK, dV
+
+
+def check_status(stream=None):
+    rc = kmip_get_status(stream)
+    if rc:
+        raise KmipError(rc, "device status")

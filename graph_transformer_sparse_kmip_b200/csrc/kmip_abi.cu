@@ -1,0 +1,180 @@
+// kmip_abi.cu -- the C ABI of libkmip (declared in include/kmip.h): argument
+// checks, the per-device status word, work-list scratch and kernel dispatch.
+#include <math.h>
+
+#include <mutex>
+
+#include "kmip_internal.h"
+
+#if defined(__GNUC__)
+#define KMIP_EXPORT extern "C" __attribute__((visibility("default")))
+#else
+#define KMIP_EXPORT extern "C"
+#endif
+
+namespace kmip {
+
+// Per-device status word: the first device-side error since the last
+// kmip_get_status() call (0 = none).
+__device__ int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_status_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+
+// Device address of g_status on the current device (resolved once per device).
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+kmip_status_t check_common(int64_t N, int H, int d, int k, float scale, kmip_dtype_t dtype) {
+  if (N < 0 || N > INT32_MAX || H < 1 || k < 1 || !(scale > 0.f) || !isfinite(scale))
+    return KMIP_ERR_INVALID_ARG;
+  if (dtype != KMIP_BF16 && dtype != KMIP_F32) return KMIP_ERR_INVALID_ARG;
+  if (H > 64 || k > 64 || !supported_d(d)) return KMIP_ERR_UNSUPPORTED;
+  if ((int64_t)N * H * (int64_t)(d > k ? d : k) > ((int64_t)1 << 40))
+    return KMIP_ERR_UNSUPPORTED;
+  return KMIP_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_sm_count[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+}  // namespace kmip
+
+using namespace kmip;
+
+KMIP_EXPORT kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void* V,
+                                        const int32_t* graph_offsets, int64_t N, int H, int d,
+                                        int k, float scale, void* out, int32_t* idx, float* lse,
+                                        kmip_stream_t stream_, int num_graphs,
+                                        kmip_dtype_t dtype) {
+  kmip_status_t st = check_common(N, H, d, k, scale, dtype);
+  if (st != KMIP_OK) return st;
+  if (graph_offsets && num_graphs < 1) return KMIP_ERR_INVALID_ARG;
+  if (N == 0) return KMIP_OK;
+  if (!Q || !K || !V || !out || !idx || !lse) return KMIP_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
+    return KMIP_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  int* status = status_ptr();
+  if (!status) return KMIP_ERR_CUDA;
+
+  const bool tc = dtype == KMIP_BF16 && fwd_tc_supported(d, k);
+  const int qpi = tc ? kTcQueries : kSimtQueries;
+  const int G = graph_offsets ? num_graphs : 1;
+  const int64_t max_items = max_work_items(N, G, qpi);
+  if (max_items * H > INT32_MAX) return KMIP_ERR_UNSUPPORTED;
+
+  // Work-list scratch: [count (16 B)] [items], stream-ordered.
+  void* scratch = nullptr;
+  const size_t bytes = 16 + sizeof(WorkItem) * (size_t)max_items;
+  if (cudaMallocAsync(&scratch, bytes, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return KMIP_ERR_CUDA;
+  }
+  int* count = static_cast<int*>(scratch);
+  WorkItem* items = reinterpret_cast<WorkItem*>(static_cast<char*>(scratch) + 16);
+
+  cudaError_t e = launch_worklist(graph_offsets, G, (int)N, qpi, items, count, (int)max_items,
+                                  status, stream);
+  if (e == cudaSuccess) {
+    FwdArgs a{Q, K, V, (int)N, H, d, k, scale, out, idx, lse, items, count, (int)max_items, status};
+    e = tc ? launch_fwd_tc(a, stream) : launch_fwd_simt(dtype, a, stream);
+  }
+  cudaError_t ef = cudaFreeAsync(scratch, stream);
+  if (e != cudaSuccess || ef != cudaSuccess) {
+    cudaGetLastError();
+    return KMIP_ERR_CUDA;
+  }
+  return KMIP_OK;
+}
+
+KMIP_EXPORT kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K,
+                                        const void* V, const int32_t* idx, const float* lse,
+                                        float* dQ, float* dK, float* dV, kmip_stream_t stream_,
+                                        int64_t N, int H, int d, int k, float scale,
+                                        kmip_dtype_t dtype) {
+  kmip_status_t st = check_common(N, H, d, k, scale, dtype);
+  if (st != KMIP_OK) return st;
+  if (N == 0) return KMIP_OK;
+  if (!dOut || !Q || !K || !V || !idx || !lse || !dQ || !dK || !dV) return KMIP_ERR_INVALID_ARG;
+  if (!aligned16(dOut) || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dQ) ||
+      !aligned16(dK) || !aligned16(dV))
+    return KMIP_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  int* status = status_ptr();
+  if (!status) return KMIP_ERR_CUDA;
+  const size_t bytes = sizeof(float) * (size_t)N * H * d;
+  cudaError_t e = cudaMemsetAsync(dK, 0, bytes, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, bytes, stream);
+  if (e == cudaSuccess) {
+    BwdArgs a{dOut, Q, K, V, idx, lse, dQ, dK, dV, (int)N, H, d, k, scale, status};
+    e = launch_bwd(dtype, a, stream);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return KMIP_ERR_CUDA;
+  }
+  return KMIP_OK;
+}
+
+KMIP_EXPORT kmip_status_t kmip_get_status(kmip_stream_t stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return KMIP_ERR_CUDA;
+  }
+  int* status = status_ptr();
+  if (!status) return KMIP_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return KMIP_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return KMIP_ERR_CUDA;
+  }
+  return static_cast<kmip_status_t>(h);
+}
+
+KMIP_EXPORT const char* kmip_error_string(kmip_status_t s) {
+  switch (s) {
+    case KMIP_OK: return "KMIP_OK: success";
+    case KMIP_ERR_INVALID_ARG: return "KMIP_ERR_INVALID_ARG: invalid argument";
+    case KMIP_ERR_UNSUPPORTED: return "KMIP_ERR_UNSUPPORTED: shape outside the supported set";
+    case KMIP_ERR_CUDA: return "KMIP_ERR_CUDA: CUDA runtime error";
+    case KMIP_ERR_BAD_OFFSETS: return "KMIP_ERR_BAD_OFFSETS: malformed graph_offsets";
+    case KMIP_ERR_TIMEOUT: return "KMIP_ERR_TIMEOUT: a device pipeline wait ran out";
+    case KMIP_ERR_BAD_INDEX: return "KMIP_ERR_BAD_INDEX: idx entry outside [-1, N)";
+  }
+  return "KMIP_ERR_UNKNOWN: unknown status code";
+}
+
+KMIP_EXPORT int kmip_version(void) { return 100; }

@@ -1,0 +1,73 @@
+// kmip_common.cuh -- small device helpers shared by the libkmip kernels.
+//
+// Element types: bf16 values widen to fp32 exactly (a bf16 is the top half of
+// an fp32), so every score and gradient here is fp32 arithmetic on exact
+// input values.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kmip.h"
+
+namespace kmip {
+
+// Work item of the forward pass: queries [q0, q1) of one graph whose keys
+// are [j0, j1).  Items are the same for every head; work index w maps to
+// head w / count and item w % count.
+struct WorkItem {
+  int q0, q1, j0, j1;
+};
+
+// Device status word handling: the first error recorded wins.
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+template <typename T>
+struct Vec;  // 16-byte vector of T, widened to fp32
+
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* f) {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      f[2 * t] = __uint_as_float(w[t] << 16);
+      f[2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
+    }
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float* f) {
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * t], f[2 * t + 1]);
+      w[t] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float* f) {
+    float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  }
+  __device__ __forceinline__ static void store(float* p, const float* f) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  }
+};
+
+// Vector reduction into fp32 global memory (sm_90+ vector form of red.add).
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+}  // namespace kmip

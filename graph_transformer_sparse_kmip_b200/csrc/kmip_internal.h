@@ -1,0 +1,66 @@
+// kmip_internal.h -- host-side launchers shared between the C ABI
+// (kmip_abi.cu) and the kernel translation units.  Not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kmip_common.cuh"
+
+namespace kmip {
+
+struct FwdArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  int N, H, d, k;
+  float scale;
+  void* out;
+  int32_t* idx;
+  float* lse;
+  const WorkItem* items;  // work list (device)
+  const int* count;       // number of items (device)
+  int max_items;          // host-side upper bound on *count
+  int* status;            // device status word
+};
+
+struct BwdArgs {
+  const void* dO;
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int32_t* idx;
+  const float* lse;
+  float* dQ;
+  float* dK;
+  float* dV;
+  int N, H, d, k;
+  float scale;
+  int* status;
+};
+
+// Queries per work item of each forward kernel.
+constexpr int kSimtQueries = 128;
+constexpr int kTcQueries = 256;
+
+// Upper bound on the number of work items for N nodes in G graphs.
+inline int64_t max_work_items(int64_t N, int64_t G, int queries_per_item) {
+  return (N + queries_per_item - 1) / queries_per_item + G;
+}
+
+cudaError_t launch_worklist(const int32_t* offsets, int G, int N, int queries_per_item,
+                            WorkItem* items, int* count, int max_items, int* status,
+                            cudaStream_t stream);
+
+cudaError_t launch_fwd_simt(kmip_dtype_t dtype, const FwdArgs& a, cudaStream_t stream);
+
+// tcgen05 forward (bf16).  Returns cudaErrorNotSupported when the shape is
+// not covered by the tensor-core kernel.
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
+bool fwd_tc_supported(int d, int k);
+
+cudaError_t launch_bwd(kmip_dtype_t dtype, const BwdArgs& a, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace kmip

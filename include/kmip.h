@@ -1,0 +1,138 @@
+/*
+ * kmip.h -- C ABI of libkmip: k-Maximum-Inner-Product (k-MIP) attention for
+ * graph transformers on NVIDIA B200 (sm_100a).
+ *
+ * The operation (k-Maximum Inner Product Attention for Graph Transformers
+ * and the Expressive Power of GraphGPS, Abstract: "selects the most relevant
+ * key nodes per query via a top-k operation", combined with a score
+ * computation whose memory is linear in the node count): for query node i
+ * of graph g and head h,
+ *
+ *   s_j  = Q[i,h,:] . K[j,h,:]          for every node j of graph g
+ *   S    = the k_eff = min(k, n_g) keys with the largest s_j
+ *          (larger s first; equal s -> smaller node index first)
+ *   lse  = log sum_{j in S} exp(scale * s_j)          (natural log)
+ *   p_j  = exp(scale * s_j - lse)
+ *   out  = sum_{j in S} p_j V[j,h,:]
+ *
+ * and its backward pass through the selected scores (the pages time a
+ * "training setting", Tables 10-12 and 16; the selection is piecewise
+ * constant and gets no gradient):
+ *
+ *   dP_j = dOut . V_j,  D = sum_j p_j dP_j,  dS_j = p_j (dP_j - D)
+ *   dQ_i = scale sum_j dS_j K_j,  dK_j += scale dS_j Q_i,  dV_j += p_j dOut_i
+ *
+ * Graphs: a batch of graphs is a block-diagonal node set.  Graph g owns the
+ * contiguous node range [graph_offsets[g], graph_offsets[g+1]); a query only
+ * ever selects keys of its own graph.  Every node of the graph, including
+ * the query node itself, is a candidate key.
+ *
+ * Memory: the N x N score matrix is never materialised; scores live in
+ * tensor memory / registers only.  The library's own device memory is a
+ * work list of O(H * (N / 128 + G)) 16-byte items per forward call, taken
+ * from the stream-ordered allocator of the current device and released on
+ * the same stream.
+ *
+ * Conventions common to every call:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device
+ *     (the device of `stream`), owned by the caller; the library keeps no
+ *     pointer after a call returns.
+ *   - Q, K, V, dOut, out are [N, H, d] row-major (node-major, heads
+ *     interleaved: the layout a Linear of width H*d produces), of the element
+ *     type `dtype`, 16-byte aligned.  idx is [N, H, k] int32, lse is [N, H]
+ *     fp32; dQ, dK, dV are [N, H, d] fp32.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).
+ *     A non-OK status returned by a call means nothing was enqueued.
+ *   - Errors found on the device (malformed graph_offsets, an index out of
+ *     range, a pipeline wait that ran out) are recorded in a per-device
+ *     status word and reported by kmip_get_status(); outputs of the affected
+ *     work are left untouched.
+ *   - Supported: N in [0, 2^31 - 1]; 1 <= H <= 64; d in {16, 32, 64, 128};
+ *     1 <= k <= 64; scale finite and > 0.
+ */
+#ifndef KMIP_H
+#define KMIP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream (a cudaStream_t); NULL means the legacy default stream. */
+typedef void* kmip_stream_t;
+
+typedef enum {
+  KMIP_BF16 = 0, /* bfloat16 inputs; scores accumulated in fp32 */
+  KMIP_F32 = 1   /* fp32 inputs; scores by fp32 fused multiply-add */
+} kmip_dtype_t;
+
+typedef enum {
+  KMIP_OK = 0,
+  KMIP_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad scale */
+  KMIP_ERR_UNSUPPORTED = 2, /* d, k or H outside the supported set */
+  KMIP_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  KMIP_ERR_BAD_OFFSETS = 4, /* device: graph_offsets not 0 = o_0 <= ... <= o_G = N */
+  KMIP_ERR_TIMEOUT = 5,     /* device: a pipeline wait ran out (kernel gave up) */
+  KMIP_ERR_BAD_INDEX = 6    /* device: idx entry outside [-1, N) in the backward */
+} kmip_status_t;
+
+/*
+ * Forward pass.
+ *   Q, K, V        [N, H, d] of `dtype` (device).
+ *   graph_offsets  int32 [num_graphs + 1] (device): offsets[0] = 0,
+ *                  offsets[num_graphs] = N, non-decreasing (empty graphs are
+ *                  allowed).  NULL means one graph of N nodes (num_graphs is
+ *                  then ignored).  Checked on the device: a malformed array
+ *                  records KMIP_ERR_BAD_OFFSETS and no output is written.
+ *   N, H, d, k     sizes; scale multiplies the scores inside the softmax
+ *                  (selection uses the unscaled scores; equivalent for scale > 0).
+ *   out            [N, H, d] of `dtype` (device), overwritten.
+ *   idx            [N, H, k] int32 (device), overwritten: the kept keys as
+ *                  global node indices, larger score first, padded with -1
+ *                  when the graph has fewer than k nodes.
+ *   lse            [N, H] fp32 (device), overwritten: log-sum-exp of the
+ *                  scaled kept scores (needed by the backward).
+ * bf16 inputs run on the tcgen05 tensor-core path (scores exact products,
+ * fp32 accumulation); fp32 inputs run an fp32 FMA path.
+ * Returns KMIP_OK, KMIP_ERR_INVALID_ARG, KMIP_ERR_UNSUPPORTED or KMIP_ERR_CUDA.
+ */
+kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void* V,
+                            const int32_t* graph_offsets, int64_t N, int H, int d, int k,
+                            float scale, void* out, int32_t* idx, float* lse,
+                            kmip_stream_t stream, int num_graphs, kmip_dtype_t dtype);
+
+/*
+ * Backward pass.
+ *   dOut           [N, H, d] of `dtype` (device): gradient of the loss w.r.t. out.
+ *   Q, K, V        the forward's inputs; idx, lse the forward's outputs.
+ *   dQ, dK, dV     [N, H, d] fp32 (device), overwritten (the library zeroes
+ *                  dK and dV itself before scattering into them).
+ * dK and dV are accumulated with fp32 atomics, so their bits may differ from
+ * run to run in the last places; dQ is deterministic.  An idx entry outside
+ * [-1, N) records KMIP_ERR_BAD_INDEX on the device and is skipped.
+ * Returns KMIP_OK, KMIP_ERR_INVALID_ARG, KMIP_ERR_UNSUPPORTED or KMIP_ERR_CUDA.
+ */
+kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K, const void* V,
+                            const int32_t* idx, const float* lse, float* dQ, float* dK,
+                            float* dV, kmip_stream_t stream, int64_t N, int H, int d, int k,
+                            float scale, kmip_dtype_t dtype);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status
+ * word (the first device-side error recorded since the last call), or
+ * KMIP_ERR_CUDA if the synchronisation itself failed.
+ */
+kmip_status_t kmip_get_status(kmip_stream_t stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* kmip_error_string(kmip_status_t status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int kmip_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KMIP_H */
