@@ -18,9 +18,9 @@ LIB_PATH = os.path.join(_PKG, "libkmip.so")
 KMIP_BF16, KMIP_F32 = 0, 1
 STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTED",
                 3: "KMIP_ERR_CUDA", 4: "KMIP_ERR_BAD_OFFSETS", 5: "KMIP_ERR_TIMEOUT",
-                6: "KMIP_ERR_BAD_INDEX"}
-EXPORTED = ("kmip_attn_fwd", "kmip_attn_bwd", "kmip_get_status", "kmip_error_string",
-            "kmip_version")
+                6: "KMIP_ERR_BAD_INDEX", 7: "KMIP_ERR_SCRATCH_LIMIT"}
+EXPORTED = ("kmip_attn_fwd", "kmip_attn_fwd_noalloc", "kmip_attn_bwd", "kmip_get_status",
+            "kmip_error_string", "kmip_version")
 
 _lib = None
 
@@ -43,6 +43,8 @@ def load() -> ctypes.CDLL:
     P, I32, I64, F32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
     lib.kmip_attn_fwd.argtypes = [P, P, P, P, I64, I32, I32, I32, F32, P, P, P, P, I32, I32]
     lib.kmip_attn_fwd.restype = I32
+    lib.kmip_attn_fwd_noalloc.argtypes = lib.kmip_attn_fwd.argtypes
+    lib.kmip_attn_fwd_noalloc.restype = I32
     lib.kmip_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, F32, I32]
     lib.kmip_attn_bwd.restype = I32
     lib.kmip_get_status.argtypes = [P]
@@ -92,6 +94,24 @@ def kmip_attn_fwd(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, stre
     return load().kmip_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N), int(H),
                                 int(d), int(k), float(scale), _ptr(out), _ptr(idx), _ptr(lse),
                                 _stream(stream), int(num_graphs), int(dtype))
+
+
+def kmip_attn_fwd_noalloc(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse,
+                          stream=None, num_graphs=None, dtype=None) -> int:
+    """kmip_attn_fwd without any device allocation inside the library: the
+    work list lives in a fixed device array of the library (for callers whose
+    memory is fully owned by their own pool, or who must not allocate after
+    start-up).  Calls on one device must not overlap on the GPU."""
+    _check_cuda(Q, K, V, graph_offsets, out, idx, lse)
+    G = (graph_offsets.numel() - 1) if graph_offsets is not None else 1
+    if num_graphs is None:
+        num_graphs = G
+    if dtype is None:
+        dtype = dtype_code(Q.dtype)
+    return load().kmip_attn_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N),
+                                        int(H), int(d), int(k), float(scale), _ptr(out),
+                                        _ptr(idx), _ptr(lse), _stream(stream), int(num_graphs),
+                                        int(dtype))
 
 
 def kmip_attn_bwd(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None, N=None, H=None, d=None,

@@ -25,6 +25,8 @@ std::mutex g_mu;
 int* g_status_ptr[kMaxDevices] = {};
 int g_sm_count[kMaxDevices] = {};
 
+}  // namespace
+
 // Device address of g_status on the current device (resolved once per device).
 int* status_ptr() {
   int dev = 0;
@@ -38,7 +40,11 @@ int* status_ptr() {
   return g_status_ptr[dev];
 }
 
+namespace {
+
 bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+}  // namespace
 
 kmip_status_t check_common(int64_t N, int H, int d, int k, float scale, kmip_dtype_t dtype) {
   if (N < 0 || N > INT32_MAX || H < 1 || k < 1 || !(scale > 0.f) || !isfinite(scale))
@@ -51,8 +57,6 @@ kmip_status_t check_common(int64_t N, int H, int d, int k, float scale, kmip_dty
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-}  // namespace
 
 int device_sm_count() {
   int dev = 0;
@@ -173,6 +177,8 @@ KMIP_EXPORT const char* kmip_error_string(kmip_status_t s) {
     case KMIP_ERR_BAD_OFFSETS: return "KMIP_ERR_BAD_OFFSETS: malformed graph_offsets";
     case KMIP_ERR_TIMEOUT: return "KMIP_ERR_TIMEOUT: a device pipeline wait ran out";
     case KMIP_ERR_BAD_INDEX: return "KMIP_ERR_BAD_INDEX: idx entry outside [-1, N)";
+    case KMIP_ERR_SCRATCH_LIMIT:
+      return "KMIP_ERR_SCRATCH_LIMIT: work list exceeds the no-allocation entry point's fixed array";
   }
   return "KMIP_ERR_UNKNOWN: unknown status code";
 }

@@ -63,4 +63,11 @@ cudaError_t launch_bwd(kmip_dtype_t dtype, const BwdArgs& a, cudaStream_t stream
 
 int device_sm_count();
 
+// Per-device status word address (nullptr if it cannot be resolved).
+int* status_ptr();
+
+// Shared argument checks of the entry points (no device access).
+kmip_status_t check_common(int64_t N, int H, int d, int k, float scale, kmip_dtype_t dtype);
+bool aligned16(const void* p);
+
 }  // namespace kmip

@@ -74,7 +74,8 @@ typedef enum {
   KMIP_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
   KMIP_ERR_BAD_OFFSETS = 4, /* device: graph_offsets not 0 = o_0 <= ... <= o_G = N */
   KMIP_ERR_TIMEOUT = 5,     /* device: a pipeline wait ran out (kernel gave up) */
-  KMIP_ERR_BAD_INDEX = 6    /* device: idx entry outside [-1, N) in the backward */
+  KMIP_ERR_BAD_INDEX = 6,   /* device: idx entry outside [-1, N) in the backward */
+  KMIP_ERR_SCRATCH_LIMIT = 7 /* kmip_attn_fwd_noalloc: work list larger than its fixed array */
 } kmip_status_t;
 
 /*
@@ -101,6 +102,38 @@ kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void* V,
                             const int32_t* graph_offsets, int64_t N, int H, int d, int k,
                             float scale, void* out, int32_t* idx, float* lse,
                             kmip_stream_t stream, int num_graphs, kmip_dtype_t dtype);
+
+/*
+ * Forward pass that allocates no device memory.  (No counterpart in the
+ * pages: this is an interface variant for callers, not part of the method.)
+ *
+ * Same arguments, outputs and results as kmip_attn_fwd.  kmip_attn_fwd
+ * takes its work list from the stream-ordered allocator on each call; this
+ * variant is for callers that cannot let a library allocate: a framework
+ * whose own memory pool already holds the GPU's memory, a driver or
+ * virtualised device without stream-ordered memory pools, or a loop that
+ * must not enter the allocator once it is running.  The work list lives in a
+ * fixed device array inside the library (about 1 MiB, held on every GPU that
+ * loads the library until the process exits); no cudaMalloc, cudaFree or
+ * allocating library routine is called.
+ *
+ * Limit: ceil(N / 256) + num_graphs <= 65536 work items for bf16 inputs on
+ * the tensor-core path, ceil(N / 128) + num_graphs <= 65536 otherwise
+ * (num_graphs counts as 1 when graph_offsets is NULL); larger calls return
+ * KMIP_ERR_SCRATCH_LIMIT with nothing enqueued.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and so should come before any stream capture.
+ * Every call on a device shares the one array and it keeps the last call's
+ * contents; nothing in it needs to be zero, since each call writes the whole
+ * work list it reads.  Calls whose work overlaps on the GPU (on different
+ * streams, or from host threads that do not order them) race on the array
+ * and must be serialised by the caller.
+ */
+kmip_status_t kmip_attn_fwd_noalloc(const void* Q, const void* K, const void* V,
+                                    const int32_t* graph_offsets, int64_t N, int H, int d,
+                                    int k, float scale, void* out, int32_t* idx, float* lse,
+                                    kmip_stream_t stream, int num_graphs, kmip_dtype_t dtype);
 
 /*
  * Backward pass.
