@@ -51,6 +51,8 @@ def load() -> ctypes.CDLL:
     lib.kmip_get_status.restype = I32
     lib.kmip_error_string.argtypes = [I32]
     lib.kmip_error_string.restype = ctypes.c_char_p
+    lib.kmip_test_wait_timeout.argtypes = [P, I32]
+    lib.kmip_test_wait_timeout.restype = I32
     lib.kmip_version.argtypes = []
     lib.kmip_version.restype = I32
     _lib = lib
@@ -139,6 +141,11 @@ def kmip_error_string(code: int) -> str:
 
 def kmip_version() -> int:
     return load().kmip_version()
+
+
+def kmip_test_wait_timeout(timeout_us: int, stream=None) -> int:
+    """Test hook (include/kmip_testing.h): a bounded wait that must run out."""
+    return load().kmip_test_wait_timeout(_stream(stream), int(timeout_us))
 
 
 # --- convenience wrappers that allocate the outputs with torch ---

@@ -39,7 +39,8 @@ struct BwdArgs {
   int* status;
 };
 
-// Queries per work item of each forward kernel.
+// Queries per work item of each forward kernel (the tensor-core forward
+// takes two 128-row Q tiles per item).
 constexpr int kSimtQueries = 128;
 constexpr int kTcQueries = 256;
 

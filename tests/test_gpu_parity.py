@@ -142,6 +142,18 @@ def test_bad_index_reported(dev):
     assert binding.kmip_get_status() == 0
 
 
+def test_bounded_wait_times_out_and_context_survives(dev):
+    import time
+    t0 = time.time()
+    assert binding.kmip_test_wait_timeout(20000) == 0   # 20 ms limit
+    assert binding.kmip_get_status() == 5               # KMIP_ERR_TIMEOUT
+    assert time.time() - t0 < 10
+    assert binding.kmip_get_status() == 0
+    inp = wl.random_case([300], H=2, d=32, dtype="bf16", seed=3)
+    res = _run(dev, inp, 15, 0.2)                       # the context still works
+    _full_compare(inp, res, 15, 0.2)
+
+
 # --- full-size workloads, in the configuration the benchmark runs ---
 
 def _large(dev, name, k=None, n_pairs=512, bwd=None):
