@@ -311,7 +311,9 @@ def run_ours(args, ws, rank, local):
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": _traffic("fwd"),
                      "peak_source": f"{peak_kind} bf16_tflops (burst)",
-                     "algorithmic_flops_per_launch": flops},
+                     "algorithmic_flops_per_launch": flops,
+                     "path": {1: "tcgen05 tensor cores", 0: "fp32 FMA"}.get(
+                         binding.kmip_fwd_path(d, k, binding.dtype_code(g["Q"].dtype)), "?")},
         "gpu_launches": 3 * args.steps,
     }
     if sweep:

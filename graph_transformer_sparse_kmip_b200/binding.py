@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTE
                 3: "KMIP_ERR_CUDA", 4: "KMIP_ERR_BAD_OFFSETS", 5: "KMIP_ERR_TIMEOUT",
                 6: "KMIP_ERR_BAD_INDEX", 7: "KMIP_ERR_SCRATCH_LIMIT"}
 EXPORTED = ("kmip_attn_fwd", "kmip_attn_fwd_noalloc", "kmip_attn_bwd", "kmip_get_status",
-            "kmip_error_string", "kmip_version")
+            "kmip_error_string", "kmip_fwd_path", "kmip_version")
 
 _lib = None
 
@@ -53,6 +53,8 @@ def load() -> ctypes.CDLL:
     lib.kmip_error_string.restype = ctypes.c_char_p
     lib.kmip_test_wait_timeout.argtypes = [P, I32]
     lib.kmip_test_wait_timeout.restype = I32
+    lib.kmip_fwd_path.argtypes = [I32, I32, I32]
+    lib.kmip_fwd_path.restype = I32
     lib.kmip_version.argtypes = []
     lib.kmip_version.restype = I32
     _lib = lib
@@ -141,6 +143,11 @@ def kmip_error_string(code: int) -> str:
 
 def kmip_version() -> int:
     return load().kmip_version()
+
+
+def kmip_fwd_path(d: int, k: int, dtype: int = KMIP_BF16) -> int:
+    """1 = tcgen05 tensor-core forward, 0 = fp32-FMA forward, -1 = unsupported."""
+    return load().kmip_fwd_path(int(d), int(k), int(dtype))
 
 
 def kmip_test_wait_timeout(timeout_us: int, stream=None) -> int:

@@ -183,4 +183,9 @@ KMIP_EXPORT const char* kmip_error_string(kmip_status_t s) {
   return "KMIP_ERR_UNKNOWN: unknown status code";
 }
 
+KMIP_EXPORT int kmip_fwd_path(int d, int k, kmip_dtype_t dtype) {
+  if (check_common(1, 1, d, k, 1.0f, dtype) != KMIP_OK) return -1;
+  return dtype == KMIP_BF16 && fwd_tc_supported(d, k) ? 1 : 0;
+}
+
 KMIP_EXPORT int kmip_version(void) { return 100; }

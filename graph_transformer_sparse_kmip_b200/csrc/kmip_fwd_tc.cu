@@ -157,96 +157,118 @@ struct RowState {
     qn = 0;
   }
 
-  // Shared-memory insertion of (s, j), s > thr, into the k real entries (keys
-  // arrive in increasing index order, so an equal score stays behind).
-  __device__ __forceinline__ void insert_smem(int k, float s, int j) {
-    constexpr int S = kEpiThreads;
-    float* L = ls + first_slot(k) * S;
-    int* J = li + first_slot(k) * S;
-    int lo = 0, hi = k - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (L[mid * S] < s) hi = mid; else lo = mid + 1;
-    }
-    for (int e = k - 1; e > lo; --e) {
-      L[e * S] = L[(e - 1) * S];
-      J[e * S] = J[(e - 1) * S];
-    }
-    L[lo * S] = s;
-    J[lo * S] = j;
-    thr = L[(k - 1) * S];
-  }
-
   // All lanes of the warp empty their queues together, oldest entry first.
-  // in_regs: hold the list in registers while draining (only where few
+  // in_regs: the list is held in registers while draining (use where few
   // other registers are live).
-  __device__ __forceinline__ void drain(int k, bool in_regs) {
-    constexpr int S = kEpiThreads;
-    const int rounds = __reduce_max_sync(0xffffffffu, qn);
-    if (rounds == 0) return;
-    if (KCAP == kRegK && in_regs) {
-      float L[kRegK];
-      int J[kRegK];
-#pragma unroll
-      for (int t = 0; t < kRegK; ++t) {
-        L[t] = ls[t * S];
-        J[t] = li[t * S];
-      }
-      for (int r = 0; r < rounds; ++r) {
-        float s = -INFINITY;
-        int j = -1;
-        if (r < qn) {
-          s = qs[r * S];
-          j = qj[r * S];
-        }
-        if (!(s > thr)) s = -INFINITY;  // no-op pass
-        if (!__any_sync(0xffffffffu, s > thr)) continue;  // nothing enters this round
-        // Compare-exchange chain: the larger value stays, the smaller moves on.
-#pragma unroll
-        for (int t = 0; t < kRegK; ++t) {
-          const bool c = s > L[t];
-          const float hi = fmaxf(L[t], s), lo = fminf(L[t], s);
-          const int jk = c ? j : J[t], jm = c ? J[t] : j;
-          L[t] = hi;
-          s = lo;
-          J[t] = jk;
-          j = jm;
-        }
-        thr = L[kRegK - 1];
-      }
-#pragma unroll
-      for (int t = 0; t < kRegK; ++t) {
-        ls[t * S] = L[t];
-        li[t * S] = J[t];
-      }
-    } else {
-      for (int r = 0; r < rounds; ++r) {
-        if (r < qn) {
-          const float s = qs[r * S];
-          if (s > thr) insert_smem(k, s, qj[r * S]);
-        }
-      }
-    }
-    qn = 0;
-    __syncwarp();
-  }
-
+  __device__ __forceinline__ void drain(int k, bool in_regs);
 };
 
-// Queue a whole 16-score group (keys jb .. jb+15) when `on`; the drain
-// compares each score with the then-current threshold.
+// Drain with the list in registers: a branch-free compare-exchange chain per
+// round (k <= kRegK lists; the k-th best is the last of kRegK slots).
+// Returns the new threshold.  Out of line so that its code exists once.
+__device__ __noinline__ float drain_regs(float* ls, int* li, const float* qs, const int* qj,
+                                         int qn, float thr) {
+  constexpr int S = kEpiThreads;
+  const int rounds = __reduce_max_sync(0xffffffffu, qn);
+  if (rounds == 0) return thr;
+  float L[kRegK];
+  int J[kRegK];
+#pragma unroll
+  for (int t = 0; t < kRegK; ++t) {
+    L[t] = ls[t * S];
+    J[t] = li[t * S];
+  }
+  for (int r = 0; r < rounds; ++r) {
+    float s = -INFINITY;
+    int j = -1;
+    if (r < qn) {
+      s = qs[r * S];
+      j = qj[r * S];
+    }
+    if (!(s > thr)) s = -INFINITY;  // no-op pass
+    if (!__any_sync(0xffffffffu, s > thr)) continue;  // nothing enters this round
+    // Compare-exchange chain: the larger value stays, the smaller moves on.
+#pragma unroll
+    for (int t = 0; t < kRegK; ++t) {
+      const bool c = s > L[t];
+      const float hi = fmaxf(L[t], s), lo = fminf(L[t], s);
+      const int jk = c ? j : J[t], jm = c ? J[t] : j;
+      L[t] = hi;
+      s = lo;
+      J[t] = jk;
+      j = jm;
+    }
+    thr = L[kRegK - 1];
+  }
+#pragma unroll
+  for (int t = 0; t < kRegK; ++t) {
+    ls[t * S] = L[t];
+    li[t * S] = J[t];
+  }
+  __syncwarp();
+  return thr;
+}
+
+// Drain by binary search and shift in shared memory over the k real entries
+// starting at slot `first` (keys arrive in increasing index order, so an
+// equal score stays behind).  Returns the new threshold.  Out of line.
+__device__ __noinline__ float drain_smem(float* ls, int* li, const float* qs, const int* qj,
+                                         int qn, float thr, int k, int first) {
+  constexpr int S = kEpiThreads;
+  const int rounds = __reduce_max_sync(0xffffffffu, qn);
+  float* L = ls + first * S;
+  int* J = li + first * S;
+  for (int r = 0; r < rounds; ++r) {
+    if (r < qn) {
+      const float s = qs[r * S];
+      if (s > thr) {
+        const int jn = qj[r * S];
+        int lo = 0, hi = k - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (L[mid * S] < s) hi = mid; else lo = mid + 1;
+        }
+        for (int e = k - 1; e > lo; --e) {
+          L[e * S] = L[(e - 1) * S];
+          J[e * S] = J[(e - 1) * S];
+        }
+        L[lo * S] = s;
+        J[lo * S] = jn;
+        thr = L[(k - 1) * S];
+      }
+    }
+  }
+  __syncwarp();
+  return thr;
+}
+
+template <int KCAP>
+__device__ __forceinline__ void RowState<KCAP>::drain(int k, bool in_regs) {
+  if (KCAP == kRegK && in_regs)
+    thr = drain_regs(ls, li, qs, qj, qn, thr);
+  else
+    thr = drain_smem(ls, li, qs, qj, qn, thr, k, first_slot(k));
+  qn = 0;
+}
+
+// Queue the scores of a 16-score group (keys jb .. jb+15) that beat the
+// row's threshold, when `on` (predicated stores; no branch per score).
 template <int KCAP>
 __device__ __forceinline__ void append_group(RowState<KCAP>& R, const float* v, int jb, bool on) {
   constexpr int S = kEpiThreads;
   if (on) {
-    float* q = R.qs + R.qn * S;
-    int* j = R.qj + R.qn * S;
+    const float t = R.thr;
+    int n = R.qn;
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
-      q[u * S] = v[u];
-      j[u * S] = jb + u;
+      const bool a = v[u] > t;
+      if (a) {
+        R.qs[n * S] = v[u];
+        R.qj[n * S] = jb + u;
+      }
+      n += a ? 1 : 0;
     }
-    R.qn += 16;
+    R.qn = n;
   }
 }
 

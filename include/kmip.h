@@ -158,6 +158,14 @@ kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K, cons
  */
 kmip_status_t kmip_get_status(kmip_stream_t stream);
 
+/*
+ * Which forward kernel kmip_attn_fwd runs for these sizes: 1 = the tcgen05
+ * tensor-core kernel (bf16 inputs whose top-k lists, queues and K ring fit
+ * in shared memory), 0 = the fp32-FMA kernel, -1 = unsupported arguments.
+ * Pure host logic; touches no device.
+ */
+int kmip_fwd_path(int d, int k, kmip_dtype_t dtype);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char* kmip_error_string(kmip_status_t status);
 

@@ -37,6 +37,14 @@ def test_exports_every_declared_symbol(lib):
     assert set(binding.EXPORTED) <= set(declared)
 
 
+def test_forward_path_query(lib):
+    assert binding.kmip_fwd_path(32, 15, binding.KMIP_BF16) == 1
+    assert binding.kmip_fwd_path(16, 15, binding.KMIP_BF16) == 1
+    assert binding.kmip_fwd_path(32, 15, binding.KMIP_F32) == 0
+    assert binding.kmip_fwd_path(48, 15, binding.KMIP_BF16) == -1
+    assert binding.kmip_fwd_path(32, 0, binding.KMIP_BF16) == -1
+
+
 def test_error_strings_and_version(lib):
     for code, name in binding.STATUS_NAMES.items():
         assert binding.kmip_error_string(code).startswith(name)
