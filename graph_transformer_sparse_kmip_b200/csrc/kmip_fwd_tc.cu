@@ -485,17 +485,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (lane == 0) mbar_arrive(smem_addr(tempty + b));
           continue;
         }
-        // Copy the row's 128 scores out and release the accumulator.
+        // Copy the row's 128 scores to registers.
         float vt[kBN / 32][32];
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) tmem_ld32(ta + c * 32, vt[c]);
         tmem_ld_wait_all();
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) reg_fence(vt[c]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(tempty + b));
-
         if (valid < kBN) {
 #pragma unroll
           for (int c = 0; c < kBN / 32; ++c)
@@ -510,15 +506,40 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (max16(vt[c] + 16) > R.thr) mask |= 1u << (2 * c + 1);
         }
         const uint32_t todo = __reduce_or_sync(0xffffffffu, mask);
-        if (todo) {
+        const bool roomy = !__any_sync(0xffffffffu, R.qn + 16 * __popc(mask) > C::kQueue);
+        if (roomy) {
+          // Common case: every lane has room for all its flagged groups, so
+          // release the accumulator now and queue from registers.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_addr(tempty + b));
 #pragma unroll
-          for (int gi = 0; gi < kBN / 16; ++gi) {
-            if (todo & (1u << gi)) {  // warp-uniform
-              if (__any_sync(0xffffffffu, R.qn > C::kQueue - 16)) R.drain(p.k, false);
+          for (int gi = 0; gi < kBN / 16; ++gi)
+            if (todo & (1u << gi))  // warp-uniform
               append_group(R, vt[gi >> 1] + (gi & 1) * 16, jt + gi * 16, (mask >> gi) & 1u);
+          __syncwarp();
+        } else {
+          // Rare: a queue could overflow.  Keep the accumulator, re-read each
+          // flagged group from tensor memory, drain between groups as needed.
+#pragma unroll 1
+          for (int gi = 0; gi < kBN / 16; ++gi) {
+            if (todo & (1u << gi)) {
+              if (__any_sync(0xffffffffu, R.qn > C::kQueue - 16)) R.drain(p.k, false);
+              float g[16];
+              tmem_ld16(ta + gi * 16, g);
+              tmem_ld_wait(g);
+#pragma unroll
+              for (int u = 0; u < 16; ++u)
+                if (gi * 16 + u >= valid) g[u] = -INFINITY;
+              append_group(R, g, jt + gi * 16, (mask >> gi) & 1u);
               __syncwarp();
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_addr(tempty + b));
+        }
+        if (todo) {
           // Insert once half the lanes have queued groups, or before a queue
           // could overflow during the next tile.
           if (__popc(__ballot_sync(0xffffffffu, R.qn > 0)) >= 16 ||
