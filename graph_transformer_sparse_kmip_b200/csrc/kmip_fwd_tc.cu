@@ -252,7 +252,10 @@ __device__ __forceinline__ void RowState<KCAP>::drain(int k, bool in_regs) {
 }
 
 // Queue the scores of a 16-score group (keys jb .. jb+15) that beat the
-// row's threshold, when `on` (predicated stores; no branch per score).
+// row's threshold, when `on`.  Branch-free: every score is written at the
+// queue tail and the tail only advances past qualifying ones (a later score
+// overwrites a rejected one).  The caller guarantees room for 16 more
+// entries, so every store stays inside the queue.
 template <int KCAP>
 __device__ __forceinline__ void append_group(RowState<KCAP>& R, const float* v, int jb, bool on) {
   constexpr int S = kEpiThreads;
@@ -261,12 +264,9 @@ __device__ __forceinline__ void append_group(RowState<KCAP>& R, const float* v, 
     int n = R.qn;
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
-      const bool a = v[u] > t;
-      if (a) {
-        R.qs[n * S] = v[u];
-        R.qj[n * S] = jb + u;
-      }
-      n += a ? 1 : 0;
+      R.qs[n * S] = v[u];
+      R.qj[n * S] = jb + u;
+      n += v[u] > t ? 1 : 0;
     }
     R.qn = n;
   }
