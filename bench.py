@@ -386,6 +386,26 @@ def run_reference(args, ws, rank):
     }
 
 
+def run_profile_calls(args):
+    """A few forward calls of the workload and nothing else: the command an
+    ncu capture of the forward kernel runs (no timing loop, no baselines)."""
+    import dataclasses
+    w = wl.WORKLOADS[args.workload]
+    if args.nodes:
+        if w.sizes_range is not None:
+            raise SystemExit("--nodes applies to single-graph workloads")
+        w = dataclasses.replace(w, N=args.nodes)
+    k = args.k or w.k
+    dev = torch.device("cuda", 0)
+    inp = wl.make_inputs(w, with_grad_out=False)
+    g = {n: t.to(dev) for n, t in inp.items()}
+    for _ in range(args.profile_calls):
+        binding.attn_fwd(g["Q"], g["K"], g["V"], k, w.scale, g["offsets"])
+    torch.cuda.synchronize()
+    binding.check_status()
+    print(json.dumps({"profile_calls": args.profile_calls, "workload": w.name, "N": w.N, "k": k}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -398,10 +418,17 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--nodes", type=int, default=None,
+                    help="override N of a single-graph workload (profiling only)")
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="run this many forward calls and exit (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = _dist()
+    if args.profile_calls:
+        run_profile_calls(args)
+        return
     if args.impl == "reference":
         res = run_reference(args, ws, rank)
         if res is not None:
