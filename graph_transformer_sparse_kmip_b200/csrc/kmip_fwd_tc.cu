@@ -5,34 +5,40 @@
 // and attends over them only; the N x N score matrix is never stored, so
 // memory stays linear in N.  Here the scores of a 256-query x 128-key tile
 // are dense contractions on the tensor cores (tcgen05, fp32 accumulators in
-// tensor memory), and the running top-k filter reads them straight out of
+// tensor memory), and a running top-k filter reads them straight out of
 // tensor memory.
 //
 // Persistent CTAs, one per SM, walk the work list (256 queries of one graph,
 // one head per item).  Warp roles:
-//   warp 0       TMA producer: the item's two 128-row Q tiles once, then the
-//                graph's K tiles (128 keys each) through a shared-memory ring.
-//   warps 1, 2   MMA issuers, one thread each, alternating K tiles: S = Q K^T
-//                for both Q tiles into the warp's own TMEM accumulator (2 x
-//                128 lanes x 128 fp32 columns).  One thread issuing every MMA,
-//                commit and wait cannot keep the tensor pipe busy when d is
-//                small (a tile is only 2 d/16 instructions); two can.
-//   warps 3..10  epilogue, one thread per query row: it copies the tile's 128
-//                scores of its row to registers and releases the accumulator
-//                at once.  The per-score filter has no branch: a three-input-
-//                max tree gives each 16-column group's maximum, and a group
-//                whose maximum beats the row's threshold (its k-th best score
-//                so far) sets a bit in a candidate mask.  The warp walks the
-//                union of flagged groups and queues each flagged lane's whole
-//                group in shared memory.  Queues are drained by all lanes
-//                together (one entry per lane per round) into the row's sorted
-//                list, held in registers while the drain runs (a branch-free
-//                compare-exchange chain for k <= 16; binary search and shift in
-//                shared memory for larger k).  The first tile of an item, where
-//                the threshold starts at -inf, is queued and drained 32 scores
-//                at a time straight from tensor memory.  After the last key
-//                tile: the softmax over the kept scores, lse, and the weighted
-//                sum of the kept V rows (16-byte loads).
+//   warp 0        TMA producer: the item's two 128-row Q tiles once, then the
+//                 graph's K tiles (128 keys each) through a shared-memory ring.
+//   warps 1, 2    MMA issuers, one thread each, alternating K tiles: S = Q K^T
+//                 for both Q tiles into the warp's own TMEM accumulator (2 x
+//                 128 lanes x 128 fp32 columns).  One thread issuing every MMA,
+//                 commit and wait cannot keep the tensor pipe busy when d is
+//                 small (a tile is only 2 d/16 instructions); two can.
+//   warps 3..10   filters, one thread per query row.  A filter copies its
+//                 row's 128 scores of the tile to registers in two halves and
+//                 hands the accumulator back at once.  The per-score test has
+//                 no branch: a three-input-max tree gives each 16-column
+//                 group's maximum, and a group whose maximum beats the row's
+//                 threshold (a lower bound of its k-th best score so far) is
+//                 stored whole, as a 16-score "record", in one of two record
+//                 buffers of the warp's rows.  A full buffer (or, once enough
+//                 rows hold records, a buffer whose twin is free) is handed
+//                 to the warp's insert warp, and the filter goes on with the
+//                 other buffer.  So the filters' work per tile is short and
+//                 even, and the accumulators turn over at the pace of the MMAs.
+//   warps 11..18  inserters, one per filter warp and one thread per row: they
+//                 take the handed-over buffers in order, insert every
+//                 recorded score that beats the row's threshold into the
+//                 row's sorted top-k list (a branch-free compare-exchange
+//                 chain over a list held in registers for k <= 16; binary
+//                 search and shift in shared memory for larger k), publish
+//                 the new threshold to the filter, and after an item's last
+//                 batch compute the softmax over the kept scores, lse, and the
+//                 weighted sum of the kept V rows (16-byte loads) while the
+//                 filters already work on the next item.
 // Keys outside the query's graph are never loaded (the key range comes from
 // the work item); the last tile of a graph masks its tail columns.
 //
@@ -54,20 +60,23 @@ using namespace sm100;
 
 constexpr int kBM = 128;           // rows of one Q tile (TMEM lanes)
 constexpr int kMT = 2;             // Q tiles per work item
+constexpr int kRows = kBM * kMT;   // query rows per work item
 constexpr int kBN = 128;           // keys per K tile (MMA N)
 constexpr int kNB = 2;             // accumulator buffers, one per MMA warp
 constexpr int kMmaWarps = kNB;
-constexpr int kEpiWarps = 8;       // 4 lane quarters x 2 Q tiles
-constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kFirstEpiWarp = 1 + kMmaWarps;
-constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
-constexpr int kRegK = 16;          // lists up to this k live in registers during a drain
+constexpr int kFilterWarps = 8;    // 4 lane quarters x 2 Q tiles
+constexpr int kInsertWarps = kFilterWarps;
+constexpr int kFirstFilterWarp = 1 + kMmaWarps;
+constexpr int kFirstInsertWarp = kFirstFilterWarp + kFilterWarps;
+constexpr int kThreads = 32 * (kFirstInsertWarp + kInsertWarps);
+constexpr int kRegK = 16;          // lists up to this k are insert-sorted in registers
+constexpr int kHandLanes = 16;      // rows holding records that hand a batch over early
 constexpr uint32_t kTmemCols = kNB * kMT * kBN;  // 512
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 constexpr size_t kSmemBudget = 227 * 1024;
 constexpr size_t kMinSmem = 120 * 1024;  // keeps one CTA (one TMEM owner) per SM
 
-static_assert(kTcQueries == kBM * kMT, "work item size");
+static_assert(kTcQueries == kRows, "work item size");
 static_assert(kTmemCols == 512, "tensor memory budget");
 
 template <int D, int KCAP>
@@ -81,18 +90,44 @@ struct Cfg {
   static constexpr int kBoxBytes = kRegions * kRegionBytes;   // a 128-row box, all of d
   static constexpr int kQBytes = kMT * kBoxBytes;             // the item's Q tiles
   static constexpr int kStageBytes = kBoxBytes;               // one K tile (128 keys)
-  static constexpr int kListBytes = 2 * KCAP * kEpiThreads * 4;
+  static constexpr int kListStride = KCAP + 1;                // list slots per row (+1: banks)
+  static constexpr int kListBytes = 2 * kListStride * kRows * 4;
+  // One record buffer: per row r records of 16 scores (+4 floats: banks),
+  // their first keys, and the row's record count.
+  static constexpr int rec_stride(int r) { return r * 16 + 4; }
+  static constexpr int buf_bytes(int r) { return kRows * (rec_stride(r) + r + 1) * 4; }
+  static constexpr int kMiscBytes = kRows * 4 + 2 * kFilterWarps * 4;  // thresholds, batch flags
   static constexpr int kBarBytes = 1024;
-  static constexpr int kBase = kQBytes + kListBytes + kBarBytes + 1024;  // + slack
-  // Candidate queue: 32 entries per row where three ring stages still fit, else 16.
-  static constexpr int kQueue =
-      (int)((kSmemBudget - kBase - 32 * 8 * kEpiThreads) / kStageBytes) >= 3 ? 32 : 16;
-  static constexpr int kFixed = kBase + kQueue * 8 * kEpiThreads;
-  static constexpr int kStagesFit = (int)((kSmemBudget - kFixed) / kStageBytes);
+  static constexpr int kBase = kQBytes + kListBytes + kMiscBytes + kBarBytes + 1024;  // + align
+  static constexpr int stages_for(int r) {
+    return ((int)kSmemBudget - kBase - 2 * buf_bytes(r)) / kStageBytes;
+  }
+  // Records per row and buffer: the most that leave four ring stages (else two).
+  static constexpr int kRec = stages_for(4) >= 4   ? 4
+                              : stages_for(3) >= 4 ? 3
+                              : stages_for(2) >= 4 ? 2
+                              : stages_for(2) >= 2 ? 2
+                                                   : 1;
+  static constexpr int kRecStride = rec_stride(kRec);
+  static constexpr int kStagesFit = stages_for(kRec);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-  static constexpr size_t kSmem = (size_t)kFixed + (size_t)kStages * kStageBytes;
+  static constexpr bool kFits = kStages >= 2;
+  // Byte offsets from the 1024-aligned base.
+  static constexpr int kOffK = kQBytes;                                  // K ring
+  static constexpr int kOffLs = kOffK + kStages * kStageBytes;           // list scores [rows][LS]
+  static constexpr int kOffLi = kOffLs + kListStride * kRows * 4;        // list keys [rows][LS]
+  static constexpr int kOffRs = kOffLi + kListStride * kRows * 4;        // [2][rows][kRecStride]
+  static constexpr int kOffRj = kOffRs + 2 * kRows * kRecStride * 4;     // [2][kRec][rows]
+  static constexpr int kOffRn = kOffRj + 2 * kRec * kRows * 4;           // [2][rows]
+  static constexpr int kOffThr = kOffRn + 2 * kRows * 4;                 // [rows]
+  static constexpr int kOffFlag = kOffThr + kRows * 4;                   // [2][filter warps]
+  static constexpr int kOffBars = kOffFlag + 2 * kFilterWarps * 4;
+  static constexpr size_t kSmem = (size_t)kOffBars + kBarBytes + 1024;
   static constexpr size_t kSmemLaunch = kSmem > kMinSmem ? kSmem : kMinSmem;
-  static constexpr bool kFits = kStages >= 2 && kSmem <= kSmemBudget;
+  static_assert(!kFits || kSmem <= kSmemBudget, "shared-memory layout");
+  static_assert(!kFits || (kOffRs % 16 == 0 && (kRecStride * 4) % 16 == 0),
+                "records are written as float4");
+  static_assert(kOffBars % 8 == 0, "mbarrier alignment");
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
   // Start-address offset (16-byte units) of K step kk (16 bf16 columns).
   static constexpr uint32_t step_off(int kk) {
@@ -121,73 +156,98 @@ __device__ __forceinline__ float max16(const float* x) {
   return fmax3(fmax3(a, b, c), fmax3(d, e, x[15]), -INFINITY);
 }
 
-// Top-k state of one query row.  The sorted list (larger score
-// first, equal scores by smaller key index) and the FIFO candidate queue live
-// column-major in shared memory (slot t at [t * kEpiThreads]).  For
-// KCAP == kRegK the list always has kRegK slots: the first kRegK - k hold +inf
-// sentinels, the k real entries follow, so the k-th best is always the last
-// slot; otherwise the k real entries are slots 0 .. k-1.  thr is the k-th best
-// score (a key must beat it to enter).
+// A row's top-k list is its line of shared memory: scores ls[0 .. KCAP-1]
+// and keys li[...], larger score first, equal scores by smaller key.  For
+// KCAP == kRegK the list always has kRegK slots: the first kRegK - k hold
+// +inf sentinels, the k real entries follow, so the k-th best is always the
+// last slot; otherwise the k real entries are slots 0 .. k-1.  Unused slots
+// hold -inf and key -1.
 template <int KCAP>
-struct RowState {
-  float* ls;
-  int* li;
-  float* qs;
-  int* qj;
-  float thr;
-  int qn;
+__device__ __forceinline__ int first_slot(int k) {
+  return KCAP == kRegK ? kRegK - k : 0;
+}
 
-  __device__ __forceinline__ int first_slot(int k) const { return KCAP == kRegK ? kRegK - k : 0; }
-
-  __device__ __forceinline__ void reset(int k) {
-    constexpr int S = kEpiThreads;
-    if (KCAP == kRegK) {
+template <int KCAP>
+__device__ __forceinline__ void list_reset(float* ls, int* li, int k) {
+  if (KCAP == kRegK) {
 #pragma unroll
-      for (int t = 0; t < kRegK; ++t) {
-        ls[t * S] = t < kRegK - k ? INFINITY : -INFINITY;
-        li[t * S] = -1;
-      }
-    } else {
-      for (int t = 0; t < k; ++t) {
-        ls[t * S] = -INFINITY;
-        li[t * S] = -1;
-      }
+    for (int t = 0; t < kRegK; ++t) {
+      ls[t] = t < kRegK - k ? INFINITY : -INFINITY;
+      li[t] = -1;
     }
-    thr = -INFINITY;
-    qn = 0;
+  } else {
+    for (int t = 0; t < k; ++t) {
+      ls[t] = -INFINITY;
+      li[t] = -1;
+    }
   }
+}
 
-  // All lanes of the warp empty their queues together, oldest entry first.
-  // in_regs: the list is held in registers while draining (use where few
-  // other registers are live).
-  __device__ __forceinline__ void drain(int k, bool in_regs);
-};
+// Bit 16 r + u is set when score u of record r beats thr.
+template <int NREC>
+__device__ __forceinline__ uint64_t record_bits(const float* rs, int rn, float thr) {
+  static_assert(NREC <= 4, "64-bit record mask");
+  uint64_t m = 0;
+#pragma unroll
+  for (int r = 0; r < NREC; ++r) {
+    if (r < rn) {
+      const float4* src = reinterpret_cast<const float4*>(rs + r * 16);
+      uint32_t b = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 x = src[q];
+        b |= (x.x > thr ? 1u : 0u) << (4 * q);
+        b |= (x.y > thr ? 1u : 0u) << (4 * q + 1);
+        b |= (x.z > thr ? 1u : 0u) << (4 * q + 2);
+        b |= (x.w > thr ? 1u : 0u) << (4 * q + 3);
+      }
+      m |= (uint64_t)b << (16 * r);
+    }
+  }
+  return m;
+}
 
-// Drain with the list in registers: a branch-free compare-exchange chain per
-// round (k <= kRegK lists; the k-th best is the last of kRegK slots).
-// Returns the new threshold.  Out of line so that its code exists once.
-__device__ __noinline__ float drain_regs(float* ls, int* li, const float* qs, const int* qj,
-                                         int qn, float thr) {
-  constexpr int S = kEpiThreads;
-  const int rounds = __reduce_max_sync(0xffffffffu, qn);
-  if (rounds == 0) return thr;
+// Next recorded score (in key order) that still beats thr; false when none
+// is left.  rj: the row's record keys, record r at rj[r * kRows].
+__device__ __forceinline__ bool next_candidate(uint64_t& m, const float* rs, const int* rj,
+                                               float thr, float& s, int& j) {
+  while (m) {
+    const int b = __ffsll((long long)m) - 1;
+    m &= m - 1;
+    const float x = rs[b];  // record b >> 4, column b & 15
+    if (x > thr) {
+      s = x;
+      j = rj[(b >> 4) * kRows] + (b & 15);
+      return true;
+    }
+  }
+  return false;
+}
+
+// Insertion for k <= kRegK: the list is held in registers and every lane
+// takes one candidate per round through a branch-free compare-exchange
+// chain.  Records are visited in key order, so an equal score stays behind
+// the entries already listed.  Returns the new threshold.  Out of line so
+// that its code exists once.
+template <int NREC>
+__device__ __noinline__ float insert_regs(float* ls, int* li, const float* rs, const int* rj,
+                                          int rn, float thr) {
+  uint64_t m = record_bits<NREC>(rs, rn, thr);
+  if (!__any_sync(0xffffffffu, m != 0)) return thr;
   float L[kRegK];
   int J[kRegK];
 #pragma unroll
   for (int t = 0; t < kRegK; ++t) {
-    L[t] = ls[t * S];
-    J[t] = li[t * S];
+    L[t] = ls[t];
+    J[t] = li[t];
   }
-  for (int r = 0; r < rounds; ++r) {
+  while (true) {
     float s = -INFINITY;
     int j = -1;
-    if (r < qn) {
-      s = qs[r * S];
-      j = qj[r * S];
-    }
-    if (!(s > thr)) s = -INFINITY;  // no-op pass
-    if (!__any_sync(0xffffffffu, s > thr)) continue;  // nothing enters this round
-    // Compare-exchange chain: the larger value stays, the smaller moves on.
+    const bool have = next_candidate(m, rs, rj, thr, s, j);
+    if (!__any_sync(0xffffffffu, have)) break;
+    // Compare-exchange chain: the larger value stays, the smaller moves on
+    // (a lane without a candidate passes -inf through, changing nothing).
 #pragma unroll
     for (int t = 0; t < kRegK; ++t) {
       const bool c = s > L[t];
@@ -202,74 +262,40 @@ __device__ __noinline__ float drain_regs(float* ls, int* li, const float* qs, co
   }
 #pragma unroll
   for (int t = 0; t < kRegK; ++t) {
-    ls[t * S] = L[t];
-    li[t * S] = J[t];
+    ls[t] = L[t];
+    li[t] = J[t];
   }
   __syncwarp();
   return thr;
 }
 
-// Drain by binary search and shift in shared memory over the k real entries
-// starting at slot `first` (keys arrive in increasing index order, so an
-// equal score stays behind).  Returns the new threshold.  Out of line.
-__device__ __noinline__ float drain_smem(float* ls, int* li, const float* qs, const int* qj,
-                                         int qn, float thr, int k, int first) {
-  constexpr int S = kEpiThreads;
-  const int rounds = __reduce_max_sync(0xffffffffu, qn);
-  float* L = ls + first * S;
-  int* J = li + first * S;
-  for (int r = 0; r < rounds; ++r) {
-    if (r < qn) {
-      const float s = qs[r * S];
-      if (s > thr) {
-        const int jn = qj[r * S];
-        int lo = 0, hi = k - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (L[mid * S] < s) hi = mid; else lo = mid + 1;
-        }
-        for (int e = k - 1; e > lo; --e) {
-          L[e * S] = L[(e - 1) * S];
-          J[e * S] = J[(e - 1) * S];
-        }
-        L[lo * S] = s;
-        J[lo * S] = jn;
-        thr = L[(k - 1) * S];
-      }
+// Insertion for larger k: binary search and shift in shared memory over the
+// k real entries starting at slot `first`, one candidate after another in
+// key order (an equal score stays behind).  Returns the new threshold.
+template <int NREC>
+__device__ __noinline__ float insert_smem(float* ls, int* li, const float* rs, const int* rj,
+                                          int rn, float thr, int k, int first) {
+  uint64_t m = record_bits<NREC>(rs, rn, thr);
+  float* L = ls + first;
+  int* J = li + first;
+  float s;
+  int jn;
+  while (next_candidate(m, rs, rj, thr, s, jn)) {
+    int lo = 0, hi = k - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (L[mid] < s) hi = mid; else lo = mid + 1;
     }
+    for (int e = k - 1; e > lo; --e) {
+      L[e] = L[e - 1];
+      J[e] = J[e - 1];
+    }
+    L[lo] = s;
+    J[lo] = jn;
+    thr = L[k - 1];
   }
   __syncwarp();
   return thr;
-}
-
-template <int KCAP>
-__device__ __forceinline__ void RowState<KCAP>::drain(int k, bool in_regs) {
-  if (KCAP == kRegK && in_regs)
-    thr = drain_regs(ls, li, qs, qj, qn, thr);
-  else
-    thr = drain_smem(ls, li, qs, qj, qn, thr, k, first_slot(k));
-  qn = 0;
-}
-
-// Queue the scores of a 16-score group (keys jb .. jb+15) that beat the
-// row's threshold, when `on`.  Branch-free: every score is written at the
-// queue tail and the tail only advances past qualifying ones (a later score
-// overwrites a rejected one).  The caller guarantees room for 16 more
-// entries, so every store stays inside the queue.
-template <int KCAP>
-__device__ __forceinline__ void append_group(RowState<KCAP>& R, const float* v, int jb, bool on) {
-  constexpr int S = kEpiThreads;
-  if (on) {
-    const float t = R.thr;
-    int n = R.qn;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      R.qs[n * S] = v[u];
-      R.qj[n * S] = jb + u;
-      n += v[u] > t ? 1 : 0;
-    }
-    R.qn = n;
-  }
 }
 
 template <int D, int KCAP>
@@ -278,18 +304,21 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               const TcParams p) {
   using C = Cfg<D, KCAP>;
   constexpr int kStages = C::kStages;
-  constexpr int S = kEpiThreads;
+  constexpr int LS = C::kListStride, RS = C::kRecStride, NR = C::kRec;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment of the swizzled tiles.
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* q_smem = base;
-  unsigned char* k_smem = q_smem + C::kQBytes;
-  float* ls = reinterpret_cast<float*>(k_smem + kStages * C::kStageBytes);
-  int* li = reinterpret_cast<int*>(ls + KCAP * S);
-  float* qs = reinterpret_cast<float*>(li + KCAP * S);
-  int* qj = reinterpret_cast<int*>(qs + C::kQueue * S);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(qj + C::kQueue * S);
+  unsigned char* k_smem = base + C::kOffK;
+  float* ls = reinterpret_cast<float*>(base + C::kOffLs);
+  int* li = reinterpret_cast<int*>(base + C::kOffLi);
+  float* rec_s = reinterpret_cast<float*>(base + C::kOffRs);
+  int* rec_j = reinterpret_cast<int*>(base + C::kOffRj);
+  int* rec_n = reinterpret_cast<int*>(base + C::kOffRn);
+  float* thr_row = reinterpret_cast<float*>(base + C::kOffThr);
+  int* bflag = reinterpret_cast<int*>(base + C::kOffFlag);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + C::kOffBars);
   uint64_t* full = bars;                  // [kStages]  K tile landed
   uint64_t* empty = full + kStages;       // [kStages]  K tile consumed by the MMAs
   uint64_t* tfull = empty + kStages;      // [kNB]      accumulator ready
@@ -297,8 +326,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   uint64_t* qfull = tempty + kNB;         // Q tile landed
   uint64_t* qempty = qfull + 1;           // Q tile no longer read (both MMA warps)
   uint64_t* mdone = qempty + 1;           // every MMA of this CTA finished
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
+  uint64_t* rfull = mdone + 1;            // [filter warps][2] record buffer handed over
+  uint64_t* rempty = rfull + 2 * kFilterWarps;  // [filter warps][2] record buffer inserted
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(rempty + 2 * kFilterWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  static_assert((2 * kStages + 2 * kNB + 3 + 4 * kFilterWarps) * 8 + 8 <= C::kBarBytes,
+                "barrier space");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -309,11 +342,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     for (int b = 0; b < kNB; ++b) {
       mbar_init(smem_addr(tfull + b), 1);
-      mbar_init(smem_addr(tempty + b), kEpiWarps);
+      mbar_init(smem_addr(tempty + b), kFilterWarps);
     }
     mbar_init(smem_addr(qfull), 1);
     mbar_init(smem_addr(qempty), kMmaWarps);
     mbar_init(smem_addr(mdone), kMmaWarps);
+    for (int b = 0; b < 2 * kFilterWarps; ++b) {
+      mbar_init(smem_addr(rfull + b), 1);
+      mbar_init(smem_addr(rempty + b), 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -376,7 +413,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     }
-  } else if (warp < kFirstEpiWarp) {
+  } else if (warp < kFirstFilterWarp) {
     // ------------------------------------------------- MMA (two warps)
     const int m = warp - 1;  // this warp's accumulator buffer and tile parity
     if (lane == 0) {
@@ -421,144 +458,201 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       while (!mbar_try_wait(smem_addr(mdone), 0) && global_ns() - t0 < p.timeout_ns) {
       }
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - kFirstEpiWarp;     // 0..7
-    const int mt = ew >> 2;                  // Q tile of this warp
+  } else if (warp < kFirstInsertWarp) {
+    // ------------------------------------------------------------- filters
+    const int f = warp - kFirstFilterWarp;   // 0..7
+    const int mt = f >> 2;                   // Q tile of this warp
     const int quarter = warp & 3;            // TMEM lanes this warp may read
-    const int row = quarter * 32 + lane;     // row within the Q tile
-    const int et = ew * 32 + lane;           // shared-memory column of this thread
-    RowState<KCAP> R{ls + et, li + et, qs + et, qj + et, -INFINITY, 0};
-    const int64_t HD = (int64_t)p.H * D;
+    const int et = f * 32 + lane;            // this row's line in the item's row arrays
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    uint64_t* my_full = rfull + 2 * f;
+    uint64_t* my_empty = rempty + 2 * f;
+    float thr = -INFINITY;                   // lower bound of the row's k-th best score
+    int rn = 0;                              // records of this row in the current buffer
+    int cb = 0;                              // buffer being filled
+    uint32_t handed0 = 0, handed1 = 0;       // batches handed over from each buffer
+    int item0 = -1, item1 = -1;              // item of each buffer's last batch
+    int item = 0;                            // items started by this warp
     uint32_t tn = 0;
     bool ok = true;
+    // Hand accumulator buffer b back to the MMA warps.
+    auto release = [&](int b) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(tempty + b));
+    };
+    // When `on`, queue the 16 scores v (keys jb .. jb+15) as the row's next
+    // record (needs rn < NR).
+    auto push_if = [&](bool on, const float* v, int jb) {
+      const uint32_t d = smem_addr(rec_s + (cb * kRows + et) * RS + rn * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_shared_v4_if(on, d + 16 * q, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      st_shared_b32_if(on, smem_addr(rec_j + (cb * NR + rn) * kRows + et), jb);
+      rn += on ? 1 : 0;
+    };
+    // Hand the current buffer to the insert warp (flags 1: the item's last
+    // batch) and switch to the other one once its previous batch has been
+    // inserted; that batch's inserter left the row's threshold in thr_row.
+    auto hand_over = [&](int flags) {
+      rec_n[cb * kRows + et] = rn;
+      if (lane == 0) bflag[cb * kFilterWarps + f] = flags;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(my_full + cb));
+      if (cb) {
+        ++handed1;
+        item1 = item;
+      } else {
+        ++handed0;
+        item0 = item;
+      }
+      cb ^= 1;
+      rn = 0;
+      const uint32_t used = cb ? handed1 : handed0;
+      if (used > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(my_empty + cb), (used - 1) & 1,
+                                               abort_flag, p.timeout_ns)))
+          ok = false;
+        else if (flags == 0 && (cb ? item1 : item0) == item)
+          thr = fmaxf(thr, *reinterpret_cast<volatile float*>(thr_row + et));
+      }
+    };
+    // The buffer not being filled holds no batch waiting to be inserted.
+    auto other_free = [&]() -> bool {
+      const uint32_t used = cb ? handed0 : handed1;
+      return used == 0 ||
+             __any_sync(0xffffffffu, mbar_test_wait(smem_addr(my_empty + (cb ^ 1)), (used - 1) & 1));
+    };
     for (int64_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
-      const int h = (int)(w / count);
       const WorkItem it = p.items[w % count];
       const bool tile_on = mt == 0 || (it.q1 - it.q0) > kBM;  // warp-uniform
-      const int i = it.q0 + mt * kBM + row;
-      R.reset(p.k);
+      ++item;
+      thr = -INFINITY;
       const int ntiles = (it.j1 - it.j0 + kBN - 1) / kBN;
       for (int t = 0; t < ntiles; ++t, ++tn) {
         const int b = (int)(tn % kNB);
         const uint32_t use = tn / kNB;
-        const bool got = __all_sync(
-            0xffffffffu, mbar_wait(smem_addr(tfull + b), use & 1, abort_flag, p.timeout_ns));
-        if (!got) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(smem_addr(tfull + b), use & 1, abort_flag, p.timeout_ns))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        if (!tile_on) {
+          release(b);
+          continue;
+        }
         const uint32_t ta = tmem + lane_base + b * (kMT * kBN) + mt * kBN;
         const int jt = it.j0 + t * kBN;            // key of column 0
         const int valid = min(kBN, it.j1 - jt);
-        if (!tile_on) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_addr(tempty + b));
-          continue;
-        }
-        if (t == 0) {
-          // The threshold starts at -inf, so the first tile holds a large share
-          // of a row's candidates: queue and drain it straight from tensor
-          // memory, then release the accumulator.
+        // Two halves of 64 columns; the accumulator goes back to the MMA
+        // warps as soon as the second half is in registers.
 #pragma unroll 1
-          for (int c = 0; c < kBN / 32; ++c) {
-            float v[32];
-            tmem_ld32(ta + c * 32, v);
-            tmem_ld_wait(v);
-            constexpr int QB = C::kQueue < 32 ? C::kQueue : 32;  // queue batch
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[2][32];
+          tmem_ld32(ta + hf * 64, v[0]);
+          tmem_ld32(ta + hf * 64 + 32, v[1]);
+          tmem_ld_wait_all();
+          reg_fence(v[0]);
+          reg_fence(v[1]);
+          if (hf == 1) release(b);
+          if (valid < kBN) {
 #pragma unroll
-            for (int sb = 0; sb < 32; sb += QB) {
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
-              for (int u = 0; u < QB; ++u) {
-                R.qs[u * S] = c * 32 + sb + u < valid ? v[sb + u] : -INFINITY;
-                R.qj[u * S] = jt + c * 32 + sb + u;
+              for (int u = 0; u < 32; ++u)
+                if (hf * 64 + c * 32 + u >= valid) v[c][u] = -INFINITY;
+          }
+          uint32_t mask = 0;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (max16(v[c]) > thr) mask |= 1u << (2 * c);
+            if (max16(v[c] + 16) > thr) mask |= 1u << (2 * c + 1);
+          }
+          const uint32_t todo = __reduce_or_sync(0xffffffffu, mask);
+          if (todo) {
+            if (!__any_sync(0xffffffffu, rn + __popc(mask) > NR)) {
+              // Every lane has room: predicated stores, no branch per group.
+#pragma unroll
+              for (int g = 0; g < 4; ++g) push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16,
+                                                  jt + hf * 64 + g * 16);
+            } else {
+              // Some lane runs out of records within this half: hand batches
+              // over between groups.
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                if (todo & (1u << g)) {  // warp-uniform
+                  if (__any_sync(0xffffffffu, rn == NR)) hand_over(0);
+                  push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16, jt + hf * 64 + g * 16);
+                }
               }
-              R.qn = QB;
-              R.drain(p.k, true);
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_addr(tempty + b));
-          continue;
         }
-        // Copy the row's 128 scores to registers.
-        float vt[kBN / 32][32];
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(ta + c * 32, vt[c]);
-        tmem_ld_wait_all();
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) reg_fence(vt[c]);
-        if (valid < kBN) {
-#pragma unroll
-          for (int c = 0; c < kBN / 32; ++c)
-#pragma unroll
-            for (int u = 0; u < 32; ++u)
-              if (c * 32 + u >= valid) vt[c][u] = -INFINITY;
-        }
-        uint32_t mask = 0;
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-          if (max16(vt[c]) > R.thr) mask |= 1u << (2 * c);
-          if (max16(vt[c] + 16) > R.thr) mask |= 1u << (2 * c + 1);
-        }
-        const uint32_t todo = __reduce_or_sync(0xffffffffu, mask);
-        const bool roomy = !__any_sync(0xffffffffu, R.qn + 16 * __popc(mask) > C::kQueue);
-        if (roomy) {
-          // Common case: every lane has room for all its flagged groups, so
-          // release the accumulator now and queue from registers.
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_addr(tempty + b));
-#pragma unroll
-          for (int gi = 0; gi < kBN / 16; ++gi)
-            if (todo & (1u << gi))  // warp-uniform
-              append_group(R, vt[gi >> 1] + (gi & 1) * 16, jt + gi * 16, (mask >> gi) & 1u);
-          __syncwarp();
-        } else {
-          // Rare: a queue could overflow.  Keep the accumulator, re-read each
-          // flagged group from tensor memory, drain between groups as needed.
-#pragma unroll 1
-          for (int gi = 0; gi < kBN / 16; ++gi) {
-            if (todo & (1u << gi)) {
-              if (__any_sync(0xffffffffu, R.qn > C::kQueue - 16)) R.drain(p.k, false);
-              float g[16];
-              tmem_ld16(ta + gi * 16, g);
-              tmem_ld_wait(g);
-#pragma unroll
-              for (int u = 0; u < 16; ++u)
-                if (gi * 16 + u >= valid) g[u] = -INFINITY;
-              append_group(R, g, jt + gi * 16, (mask >> gi) & 1u);
-              __syncwarp();
-            }
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_addr(tempty + b));
-        }
-        if (todo) {
-          // Insert once half the lanes have queued groups, or before a queue
-          // could overflow during the next tile.
-          if (__popc(__ballot_sync(0xffffffffu, R.qn > 0)) >= 16 ||
-              __any_sync(0xffffffffu, 2 * R.qn > C::kQueue))
-            R.drain(p.k, true);
-        }
+        if (!ok) break;
+        // Hand a batch over early once enough rows hold records and the
+        // insert warp has nothing else queued.
+        if (__popc(__ballot_sync(0xffffffffu, rn > 0)) >= kHandLanes && other_free())
+          hand_over(0);
       }
       if (!ok) break;
-      R.drain(p.k, true);
+      hand_over(1);  // the item's last batch
+    }
+  } else {
+    // ----------------------------------------------------------- inserters
+    const int f = warp - kFirstInsertWarp;             // paired filter warp f
+    const int mt = f >> 2;
+    const int quarter = (f + kFirstFilterWarp) & 3;    // that filter's lane quarter
+    const int row = quarter * 32 + lane;               // row within the Q tile
+    const int et = f * 32 + lane;
+    float* L = ls + et * LS;
+    int* J = li + et * LS;
+    uint64_t* my_full = rfull + 2 * f;
+    uint64_t* my_empty = rempty + 2 * f;
+    const int64_t HD = (int64_t)p.H * D;
+    int cb = 0;
+    uint32_t taken0 = 0, taken1 = 0;  // batches taken from each buffer
+    bool ok = true;
+    for (int64_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      const int h = (int)(w / count);
+      const WorkItem it = p.items[w % count];
+      const bool tile_on = mt == 0 || (it.q1 - it.q0) > kBM;
+      const int i = it.q0 + mt * kBM + row;
+      list_reset<KCAP>(L, J, p.k);
+      float thr = -INFINITY;
+      for (;;) {
+        const uint32_t tk = cb ? taken1 : taken0;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(smem_addr(my_full + cb), tk & 1, abort_flag, p.timeout_ns))) {
+          ok = false;
+          break;
+        }
+        const int rn = rec_n[cb * kRows + et];
+        const int flags = bflag[cb * kFilterWarps + f];
+        const float* rs = rec_s + (cb * kRows + et) * RS;
+        const int* rj = rec_j + cb * NR * kRows + et;
+        if (KCAP == kRegK)
+          thr = insert_regs<NR>(L, J, rs, rj, rn, thr);
+        else
+          thr = insert_smem<NR>(L, J, rs, rj, rn, thr, p.k, first_slot<KCAP>(p.k));
+        *reinterpret_cast<volatile float*>(thr_row + et) = thr;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(my_empty + cb));
+        if (cb) ++taken1; else ++taken0;
+        cb ^= 1;
+        if (flags & 1) break;
+      }
+      if (!ok) break;
       if (tile_on && i < it.q1) {
-        const float* L = R.ls + R.first_slot(p.k) * S;
-        const int* J = R.li + R.first_slot(p.k) * S;
+        const float* Lf = L + first_slot<KCAP>(p.k);
+        const int* Jf = J + first_slot<KCAP>(p.k);
         int cnt = 0;
-        while (cnt < p.k && J[cnt * S] >= 0) ++cnt;
+        while (cnt < p.k && Jf[cnt] >= 0) ++cnt;
         // Softmax over the kept scaled scores, lse, weighted sum of V rows.
         const int64_t rowg = (int64_t)i * p.H + h;
-        const float mx = p.scale * L[0];
+        const float mx = p.scale * Lf[0];
         float sum = 0.f;
-        for (int t = 0; t < cnt; ++t) sum += expf(p.scale * L[t * S] - mx);
+        for (int t = 0; t < cnt; ++t) sum += expf(p.scale * Lf[t] - mx);
         const float lse_v = mx + logf(sum);
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -567,20 +661,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
           for (int u = 0; u < CW; ++u) o[u] = 0.f;
           for (int t = 0; t < cnt; ++t) {
-            const float pw = expf(p.scale * L[t * S] - lse_v);
-            const __nv_bfloat16* vr = p.V + (int64_t)J[t * S] * HD + h * D + c0;
+            const float pw = expf(p.scale * Lf[t] - lse_v);
+            const __nv_bfloat16* vr = p.V + (int64_t)Jf[t] * HD + h * D + c0;
 #pragma unroll
             for (int u = 0; u < CW; u += 8) {
-              float f[8];
-              Vec<__nv_bfloat16>::load(vr + u, f);
+              float fv[8];
+              Vec<__nv_bfloat16>::load(vr + u, fv);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) o[u + e] = fmaf(pw, f[e], o[u + e]);
+              for (int e = 0; e < 8; ++e) o[u + e] = fmaf(pw, fv[e], o[u + e]);
             }
           }
 #pragma unroll
           for (int u = 0; u < CW; u += 8) Vec<__nv_bfloat16>::store(p.out + rowg * D + c0 + u, o + u);
         }
-        for (int t = 0; t < p.k; ++t) p.idx[rowg * p.k + t] = t < cnt ? J[t * S] : -1;
+        for (int t = 0; t < p.k; ++t) p.idx[rowg * p.k + t] = t < cnt ? Jf[t] : -1;
         p.lse[rowg] = lse_v;
       }
     }
@@ -678,8 +772,8 @@ bool fits_d(int k) {
   return Cfg<D, 64>::kFits;
 }
 
-// Shapes whose lists, queues, Q tile and at least two K stages fit in shared
-// memory (d = 128 does not); other shapes run the fp32-FMA forward.
+// Shapes whose lists, record buffers, Q tiles and at least two K stages fit
+// in shared memory; other shapes run the fp32-FMA forward.
 bool fwd_tc_supported(int d, int k) {
   if (k < 1 || k > 64) return false;
   switch (d) {

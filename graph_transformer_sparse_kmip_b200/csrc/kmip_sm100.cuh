@@ -56,6 +56,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of whether the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // try_wait that lets the hardware suspend the thread (up to suspend_ns)
 // until the phase completes, instead of spinning on the issue slots.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
@@ -87,6 +99,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       return false;
     }
   }
+}
+
+// ---------------------------------------------------- predicated stores
+// Shared-memory stores that take effect only when `on`: a predicate, not a
+// branch, so lanes that store and lanes that do not stay converged.
+__device__ __forceinline__ void st_shared_v4_if(bool on, uint32_t addr, float a, float b, float c,
+                                                float d) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t"
+      "@q st.shared.v4.f32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"((int)on),
+      "r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+      : "memory");
+}
+
+__device__ __forceinline__ void st_shared_b32_if(bool on, uint32_t addr, int v) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %0, 0;\n\t@q st.shared.b32 [%1], %2;\n\t}" ::"r"(
+          (int)on),
+      "r"(addr), "r"(v)
+      : "memory");
 }
 
 // -------------------------------------------------------------------- TMA
