@@ -17,9 +17,10 @@
 //                 128 lanes x 128 fp32 columns).  One thread issuing every MMA,
 //                 commit and wait cannot keep the tensor pipe busy when d is
 //                 small (a tile is only 2 d/16 instructions); two can.
-//   warps 3..10   filters, one thread per query row.  A filter copies its
-//                 row's 128 scores of the tile to registers in two halves and
-//                 hands the accumulator back at once.  The per-score test has
+//   warp 3        spare (completes the first warpgroup).
+//   warps 4..11   filters, one thread per query row.  A filter copies its
+//                 row's 128 scores of the tile to registers and hands the
+//                 accumulator back at once.  The per-score test has
 //                 no branch: a three-input-max tree gives each 16-column
 //                 group's maximum, and a group whose maximum beats the row's
 //                 threshold (a lower bound of its k-th best score so far) is
@@ -29,7 +30,7 @@
 //                 to the warp's insert warp, and the filter goes on with the
 //                 other buffer.  So the filters' work per tile is short and
 //                 even, and the accumulators turn over at the pace of the MMAs.
-//   warps 11..18  inserters, one per filter warp and one thread per row: they
+//   warps 12..19  inserters, one per filter warp and one thread per row: they
 //                 take the handed-over buffers in order, insert every
 //                 recorded score that beats the row's threshold into the
 //                 row's sorted top-k list (a branch-free compare-exchange
@@ -39,6 +40,9 @@
 //                 batch compute the softmax over the kept scores, lse, and the
 //                 weighted sum of the kept V rows (16-byte loads) while the
 //                 filters already work on the next item.
+// The warpgroups rebalance their registers at the start (setmaxnreg): the
+// producer/MMA warpgroup and the inserters give some up, and the filters,
+// which hold a tile's scores, take them.
 // Keys outside the query's graph are never loaded (the key range comes from
 // the work item); the last tile of a graph masks its tail columns.
 //
@@ -66,7 +70,7 @@ constexpr int kNB = 2;             // accumulator buffers, one per MMA warp
 constexpr int kMmaWarps = kNB;
 constexpr int kFilterWarps = 8;    // 4 lane quarters x 2 Q tiles
 constexpr int kInsertWarps = kFilterWarps;
-constexpr int kFirstFilterWarp = 1 + kMmaWarps;
+constexpr int kFirstFilterWarp = 4;   // warps 0..3: producer, MMA x2, spare (one warpgroup)
 constexpr int kFirstInsertWarp = kFirstFilterWarp + kFilterWarps;
 constexpr int kThreads = 32 * (kFirstInsertWarp + kInsertWarps);
 constexpr int kRegK = 16;          // lists up to this k are insert-sorted in registers
@@ -75,6 +79,14 @@ constexpr uint32_t kTmemCols = kNB * kMT * kBN;  // 512
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 constexpr size_t kSmemBudget = 227 * 1024;
 constexpr size_t kMinSmem = 120 * 1024;  // keeps one CTA (one TMEM owner) per SM
+// Registers per thread: at launch, and after the warpgroups rebalance them
+// (producer/MMA warpgroup and inserters give some up, filters take them).
+constexpr int kLaunchRegs = 96;
+constexpr int kRegsCtl = 40, kRegsFilter = 152, kRegsInsert = 64;
+static_assert(kThreads % 128 == 0, "whole warpgroups");
+static_assert(128 * kRegsCtl + 32 * kFilterWarps * kRegsFilter + 32 * kInsertWarps * kRegsInsert <=
+                  kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 
 static_assert(kTcQueries == kRows, "work item size");
 static_assert(kTmemCols == 512, "tensor memory budget");
@@ -230,7 +242,7 @@ __device__ __forceinline__ bool next_candidate(uint64_t& m, const float* rs, con
 // the entries already listed.  Returns the new threshold.  Out of line so
 // that its code exists once.
 template <int NREC>
-__device__ __noinline__ float insert_regs(float* ls, int* li, const float* rs, const int* rj,
+__device__ __forceinline__ float insert_regs(float* ls, int* li, const float* rs, const int* rj,
                                           int rn, float thr) {
   uint64_t m = record_bits<NREC>(rs, rn, thr);
   if (!__any_sync(0xffffffffu, m != 0)) return thr;
@@ -273,7 +285,7 @@ __device__ __noinline__ float insert_regs(float* ls, int* li, const float* rs, c
 // k real entries starting at slot `first`, one candidate after another in
 // key order (an equal score stays behind).  Returns the new threshold.
 template <int NREC>
-__device__ __noinline__ float insert_smem(float* ls, int* li, const float* rs, const int* rj,
+__device__ __forceinline__ float insert_smem(float* ls, int* li, const float* rs, const int* rj,
                                           int rn, float thr, int k, int first) {
   uint64_t m = record_bits<NREC>(rs, rn, thr);
   float* L = ls + first;
@@ -368,7 +380,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int count = *p.count;
   const int64_t total = (int64_t)p.H * count;
 
-  if (warp == 0) {
+  if (warp < kFirstFilterWarp) {
+   reg_dealloc<kRegsCtl>();
+   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t kn = 0, qn = 0;  // K tiles and Q tiles issued
@@ -413,7 +427,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     }
-  } else if (warp < kFirstFilterWarp) {
+  } else if (warp <= kMmaWarps) {
     // ------------------------------------------------- MMA (two warps)
     const int m = warp - 1;  // this warp's accumulator buffer and tile parity
     if (lane == 0) {
@@ -458,7 +472,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       while (!mbar_try_wait(smem_addr(mdone), 0) && global_ns() - t0 < p.timeout_ns) {
       }
     }
+   }  // warp 3: spare
   } else if (warp < kFirstInsertWarp) {
+    reg_alloc<kRegsFilter>();
     // ------------------------------------------------------------- filters
     const int f = warp - kFirstFilterWarp;   // 0..7
     const int mt = f >> 2;                   // Q tile of this warp
@@ -545,46 +561,43 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const uint32_t ta = tmem + lane_base + b * (kMT * kBN) + mt * kBN;
         const int jt = it.j0 + t * kBN;            // key of column 0
         const int valid = min(kBN, it.j1 - jt);
-        // Two halves of 64 columns; the accumulator goes back to the MMA
-        // warps as soon as the second half is in registers.
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          float v[2][32];
-          tmem_ld32(ta + hf * 64, v[0]);
-          tmem_ld32(ta + hf * 64 + 32, v[1]);
-          tmem_ld_wait_all();
-          reg_fence(v[0]);
-          reg_fence(v[1]);
-          if (hf == 1) release(b);
-          if (valid < kBN) {
+        // The row's 128 scores in registers; the accumulator goes back to
+        // the MMA warps at once.
+        float v[kBN / 32][32];
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(ta + c * 32, v[c]);
+        tmem_ld_wait_all();
 #pragma unroll
-              for (int u = 0; u < 32; ++u)
-                if (hf * 64 + c * 32 + u >= valid) v[c][u] = -INFINITY;
-          }
-          uint32_t mask = 0;
+        for (int c = 0; c < kBN / 32; ++c) reg_fence(v[c]);
+        release(b);
+        if (valid < kBN) {
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            if (max16(v[c]) > thr) mask |= 1u << (2 * c);
-            if (max16(v[c] + 16) > thr) mask |= 1u << (2 * c + 1);
-          }
-          const uint32_t todo = __reduce_or_sync(0xffffffffu, mask);
-          if (todo) {
-            if (!__any_sync(0xffffffffu, rn + __popc(mask) > NR)) {
-              // Every lane has room: predicated stores, no branch per group.
+          for (int c = 0; c < kBN / 32; ++c)
 #pragma unroll
-              for (int g = 0; g < 4; ++g) push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16,
-                                                  jt + hf * 64 + g * 16);
-            } else {
-              // Some lane runs out of records within this half: hand batches
-              // over between groups.
+            for (int u = 0; u < 32; ++u)
+              if (c * 32 + u >= valid) v[c][u] = -INFINITY;
+        }
+        uint32_t mask = 0;
 #pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                if (todo & (1u << g)) {  // warp-uniform
-                  if (__any_sync(0xffffffffu, rn == NR)) hand_over(0);
-                  push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16, jt + hf * 64 + g * 16);
-                }
+        for (int c = 0; c < kBN / 32; ++c) {
+          if (max16(v[c]) > thr) mask |= 1u << (2 * c);
+          if (max16(v[c] + 16) > thr) mask |= 1u << (2 * c + 1);
+        }
+        const uint32_t todo = __reduce_or_sync(0xffffffffu, mask);
+        if (todo) {
+          if (!__any_sync(0xffffffffu, rn + __popc(mask) > NR)) {
+            // Every lane has room: predicated stores, no branch per group.
+#pragma unroll
+            for (int g = 0; g < kBN / 16; ++g)
+              push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16, jt + g * 16);
+          } else {
+            // Some lane runs out of records within this tile: hand batches
+            // over between groups.
+#pragma unroll
+            for (int g = 0; g < kBN / 16; ++g) {
+              if (todo & (1u << g)) {  // warp-uniform
+                if (__any_sync(0xffffffffu, rn == NR)) hand_over(0);
+                push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16, jt + g * 16);
               }
             }
           }
@@ -599,6 +612,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       hand_over(1);  // the item's last batch
     }
   } else {
+    reg_dealloc<kRegsInsert>();
     // ----------------------------------------------------------- inserters
     const int f = warp - kFirstInsertWarp;             // paired filter warp f
     const int mt = f >> 2;
@@ -738,6 +752,11 @@ cudaError_t launch_cfg(const FwdArgs& a, cudaStream_t stream) {
   if (!make_map<D>(&mq, a.Q, a.N, a.H) || !make_map<D>(&mk, a.K, a.N, a.H))
     return cudaErrorInvalidValue;
   auto kern = fwd_tc_kernel<D, KCAP>;
+  // The warpgroups' register split draws on the launch allocation: refuse
+  // to launch a build whose kernel was given fewer registers.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+  if (fa.numRegs < kLaunchRegs) return cudaErrorNotSupported;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemLaunch);
   if (e != cudaSuccess) return e;

@@ -101,6 +101,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// ------------------------------------------------------------ registers
+// Warpgroup-wide register re-allocation (every thread of the warpgroup
+// executes the same one).  inc waits until the registers are free.
+template <uint32_t R>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 // ---------------------------------------------------- predicated stores
 // Shared-memory stores that take effect only when `on`: a predicate, not a
 // branch, so lanes that store and lanes that do not stay converged.
