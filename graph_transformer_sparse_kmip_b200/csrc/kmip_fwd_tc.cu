@@ -108,7 +108,7 @@ struct Cfg {
   // their first keys, and the row's record count.
   static constexpr int rec_stride(int r) { return r * 16 + 4; }
   static constexpr int buf_bytes(int r) { return kRows * (rec_stride(r) + r + 1) * 4; }
-  static constexpr int kMiscBytes = kRows * 4 + 2 * kFilterWarps * 4;  // thresholds, batch flags
+  static constexpr int kMiscBytes = kRows * 8 + 2 * kFilterWarps * 4;  // thresholds, batch flags
   static constexpr int kBarBytes = 1024;
   static constexpr int kBase = kQBytes + kListBytes + kMiscBytes + kBarBytes + 1024;  // + align
   static constexpr int stages_for(int r) {
@@ -131,8 +131,8 @@ struct Cfg {
   static constexpr int kOffRs = kOffLi + kListStride * kRows * 4;        // [2][rows][kRecStride]
   static constexpr int kOffRj = kOffRs + 2 * kRows * kRecStride * 4;     // [2][kRec][rows]
   static constexpr int kOffRn = kOffRj + 2 * kRec * kRows * 4;           // [2][rows]
-  static constexpr int kOffThr = kOffRn + 2 * kRows * 4;                 // [rows]
-  static constexpr int kOffFlag = kOffThr + kRows * 4;                   // [2][filter warps]
+  static constexpr int kOffThr = kOffRn + 2 * kRows * 4;                 // [rows] (thr, item)
+  static constexpr int kOffFlag = kOffThr + kRows * 8;                   // [2][filter warps]
   static constexpr int kOffBars = kOffFlag + 2 * kFilterWarps * 4;
   static constexpr size_t kSmem = (size_t)kOffBars + kBarBytes + 1024;
   static constexpr size_t kSmemLaunch = kSmem > kMinSmem ? kSmem : kMinSmem;
@@ -368,6 +368,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
   }
+  // Published thresholds start as (-inf, item 0); items count from 1, so a
+  // value left in shared memory by an earlier kernel is never taken.
+  for (int r = threadIdx.x; r < kRows; r += blockDim.x)
+    reinterpret_cast<unsigned long long*>(thr_row)[r] = __float_as_uint(-INFINITY);
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_holder), kTmemCols);
     tmem_relinquish();
@@ -487,7 +491,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     int rn = 0;                              // records of this row in the current buffer
     int cb = 0;                              // buffer being filled
     uint32_t handed0 = 0, handed1 = 0;       // batches handed over from each buffer
-    int item0 = -1, item1 = -1;              // item of each buffer's last batch
     int item = 0;                            // items started by this warp
     uint32_t tn = 0;
     bool ok = true;
@@ -509,19 +512,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     };
     // Hand the current buffer to the insert warp (flags 1: the item's last
     // batch) and switch to the other one once its previous batch has been
-    // inserted; that batch's inserter left the row's threshold in thr_row.
+    // inserted.
     auto hand_over = [&](int flags) {
       rec_n[cb * kRows + et] = rn;
       if (lane == 0) bflag[cb * kFilterWarps + f] = flags;
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(my_full + cb));
-      if (cb) {
-        ++handed1;
-        item1 = item;
-      } else {
-        ++handed0;
-        item0 = item;
-      }
+      if (cb) ++handed1; else ++handed0;
       cb ^= 1;
       rn = 0;
       const uint32_t used = cb ? handed1 : handed0;
@@ -529,8 +526,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(my_empty + cb), (used - 1) & 1,
                                                abort_flag, p.timeout_ns)))
           ok = false;
-        else if (flags == 0 && (cb ? item1 : item0) == item)
-          thr = fmaxf(thr, *reinterpret_cast<volatile float*>(thr_row + et));
       }
     };
     // The buffer not being filled holds no batch waiting to be inserted.
@@ -557,6 +552,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (!tile_on) {
           release(b);
           continue;
+        }
+        {
+          // The threshold the insert warp reached for this row, if it is
+          // working on this item already.
+          const unsigned long long tv =
+              *reinterpret_cast<volatile unsigned long long*>(thr_row + 2 * et);
+          if ((int)(tv >> 32) == item) thr = fmaxf(thr, __uint_as_float((unsigned)tv));
         }
         const uint32_t ta = tmem + lane_base + b * (kMT * kBN) + mt * kBN;
         const int jt = it.j0 + t * kBN;            // key of column 0
@@ -626,6 +628,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int64_t HD = (int64_t)p.H * D;
     int cb = 0;
     uint32_t taken0 = 0, taken1 = 0;  // batches taken from each buffer
+    int item_no = 0;
     bool ok = true;
     for (int64_t w = blockIdx.x; w < total && ok; w += gridDim.x) {
       const int h = (int)(w / count);
@@ -634,6 +637,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const int i = it.q0 + mt * kBM + row;
       list_reset<KCAP>(L, J, p.k);
       float thr = -INFINITY;
+      ++item_no;
       for (;;) {
         const uint32_t tk = cb ? taken1 : taken0;
         if (!__all_sync(0xffffffffu,
@@ -649,7 +653,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           thr = insert_regs<NR>(L, J, rs, rj, rn, thr);
         else
           thr = insert_smem<NR>(L, J, rs, rj, rn, thr, p.k, first_slot<KCAP>(p.k));
-        *reinterpret_cast<volatile float*>(thr_row + et) = thr;
+        {
+          // Publish the row's threshold with the item it belongs to, in one
+          // 8-byte store, for the filter to raise its own.
+          *reinterpret_cast<volatile unsigned long long*>(thr_row + 2 * et) =
+              ((unsigned long long)(unsigned)item_no << 32) | __float_as_uint(thr);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(my_empty + cb));
         if (cb) ++taken1; else ++taken0;
