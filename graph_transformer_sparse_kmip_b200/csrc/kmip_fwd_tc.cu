@@ -788,6 +788,7 @@ template <int D>
 cudaError_t launch_d(const FwdArgs& a, cudaStream_t stream) {
   if (a.k <= kRegK) return launch_k<D, kRegK>(a, stream);
   if (a.k <= 32) return launch_k<D, 32>(a, stream);
+  if (a.k <= 48) return launch_k<D, 48>(a, stream);
   return launch_k<D, 64>(a, stream);
 }
 
@@ -797,6 +798,7 @@ template <int D>
 bool fits_d(int k) {
   if (k <= kRegK) return Cfg<D, kRegK>::kFits;
   if (k <= 32) return Cfg<D, 32>::kFits;
+  if (k <= 48) return Cfg<D, 48>::kFits;
   return Cfg<D, 64>::kFits;
 }
 

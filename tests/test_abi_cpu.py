@@ -42,6 +42,11 @@ def test_forward_path_query(lib):
     assert binding.kmip_fwd_path(16, 15, binding.KMIP_BF16) == 1
     assert binding.kmip_fwd_path(32, 15, binding.KMIP_F32) == 0
     assert binding.kmip_fwd_path(48, 15, binding.KMIP_BF16) == -1
+    # Shapes whose lists, record buffers, Q tiles and two K stages fit in
+    # shared memory take the tensor-core kernel; the rest the FMA kernel.
+    for d, k, path in [(16, 64, 1), (32, 45, 1), (32, 64, 1), (64, 32, 1), (64, 45, 1),
+                       (64, 64, 0), (128, 16, 1), (128, 17, 0), (128, 64, 0)]:
+        assert binding.kmip_fwd_path(d, k, binding.KMIP_BF16) == path, (d, k)
     assert binding.kmip_fwd_path(32, 0, binding.KMIP_BF16) == -1
 
 
