@@ -28,15 +28,16 @@
 //                 buffers of the warp's rows.  A full buffer (or, once enough
 //                 rows hold records, a buffer whose twin is free) is handed
 //                 to the warp's insert warp, and the filter goes on with the
-//                 other buffer.  So the filters' work per tile is short and
-//                 even, and the accumulators turn over at the pace of the MMAs.
+//                 other buffer; it waits for an insertion only when both of
+//                 its buffers are full.
 //   warps 12..19  inserters, one per filter warp and one thread per row: they
 //                 take the handed-over buffers in order, insert every
 //                 recorded score that beats the row's threshold into the
 //                 row's sorted top-k list (a branch-free compare-exchange
 //                 chain over a list held in registers for k <= 16; binary
-//                 search and shift in shared memory for larger k), publish
-//                 the new threshold to the filter, and after an item's last
+//                 search and shift in shared memory for larger k; lists of
+//                 16, 32, 48 or 64 slots), publish the new threshold, which
+//                 the filter reads every tile, and after an item's last
 //                 batch compute the softmax over the kept scores, lse, and the
 //                 weighted sum of the kept V rows (16-byte loads) while the
 //                 filters already work on the next item.
