@@ -49,6 +49,29 @@ def _dist():
     return ws, rank, local
 
 
+def rank_inputs(w, rank: int):
+    """This rank's batch: the workload's inputs drawn with a rank-specific
+    seed, so ranks work on independent batches (weak scaling)."""
+    return wl.make_inputs(w, with_grad_out=True, seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(vals, ws: int, device):
+    """Element-wise maximum of per-rank timings (the slowest rank sets the
+    job's time); the identity for one rank."""
+    vals = [float(v) for v in vals]
+    if ws == 1:
+        return vals
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_rank: int, ws: int, ms_per_step: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest
+    rank's time per step."""
+    return units_per_rank * ws / (ms_per_step * 1e-3)
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -153,7 +176,7 @@ def run_ours(args, ws, rank, local):
     binding.load()
     w = wl.WORKLOADS[args.workload]
     k = args.k or w.k
-    inp = wl.make_inputs(w, with_grad_out=True, seed=w.seed + 7919 * rank)
+    inp = rank_inputs(w, rank)
     N, H, d = inp["Q"].shape
     scale = w.scale
     g = {n: t.to(dev) for n, t in inp.items()}
@@ -203,16 +226,11 @@ def run_ours(args, ws, rank, local):
     binding.check_status()
     fwd_ms = [a.elapsed_time(m) for a, m, _ in evs]
     tot_ms = [a.elapsed_time(b) for a, _, b in evs]
-    t_fwd, t_tot = sum(fwd_ms), sum(tot_ms)
-    if ws > 1:
-        t = torch.tensor([t_fwd, t_tot], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_fwd, t_tot = t.tolist()
+    t_fwd, t_tot = max_over_ranks([sum(fwd_ms), sum(tot_ms)], ws, dev)
     ms_step = t_tot / args.steps
     ms_fwd = t_fwd / args.steps
-    units = N * H * ws
-    value = units / (ms_step * 1e-3)
-    fwd_value = units / (ms_fwd * 1e-3)
+    value = job_throughput(N * H, ws, ms_step)
+    fwd_value = job_throughput(N * H, ws, ms_fwd)
 
     peaks, peak_kind = _peaks()
     flops = _score_flops(inp["offsets"], H, d)
@@ -284,13 +302,9 @@ def run_ours(args, ws, rank, local):
             e2e_step()
         e_b.record(stream)
         torch.cuda.synchronize()
-        t_e2e = e_a.elapsed_time(e_b)
-        if ws > 1:
-            t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            t_e2e = t.item()
+        t_e2e = max_over_ranks([e_a.elapsed_time(e_b)], ws, dev)[0]
         binding.check_status()
-        e2e = {"value": units / (t_e2e / args.steps * 1e-3), "unit": UNIT,
+        e2e = {"value": job_throughput(N * H, ws, t_e2e / args.steps), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": t_e2e / args.steps}
 
