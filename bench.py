@@ -263,50 +263,79 @@ def run_ours(args, ws, rank, local):
                               "ms_fwd_bwd": round(statistics.mean(t[1] for t in times), 4)}
         binding.check_status()
 
-    # end to end through the public API: pinned host inputs in, host results out
+    # end to end through the public API: pinned host inputs in, host results out.
+    # Steps are pipelined the way a serving loop runs them: two slots of device
+    # buffers and three streams, so step s+1's host-to-device copy and step
+    # s-1's device-to-host copy overlap step s's kernels; every step still
+    # copies its own inputs in and its own results out.
     e2e = None
     if args.e2e:
         hostin = {n: inp[n].pin_memory() for n in ("Q", "K", "V", "dO")}
         off_h = inp["offsets"].pin_memory()
-        hostout = {"out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
-                   "idx": torch.empty(idx.shape, dtype=idx.dtype).pin_memory(),
-                   "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory(),
-                   "dQ": torch.empty(dQ.shape, dtype=dQ.dtype).pin_memory(),
-                   "dK": torch.empty(dK.shape, dtype=dK.dtype).pin_memory(),
-                   "dV": torch.empty(dV.shape, dtype=dV.dtype).pin_memory()}
-        dbuf = {n: torch.empty_like(g[n]) for n in ("Q", "K", "V", "dO")}
-        doff = torch.empty_like(g["offsets"])
+        outs = {"out": out, "idx": idx, "lse": lse, "dQ": dQ, "dK": dK, "dV": dV}
+        hostout = [{n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in outs.items()}
+                   for _ in range(2)]
+        dIn = [{n: torch.empty_like(g[n]) for n in ("Q", "K", "V", "dO")} for _ in range(2)]
+        dOff = [torch.empty_like(g["offsets"]) for _ in range(2)]
+        dOut = [outs, {n: torch.empty_like(t) for n, t in outs.items()}]
         h2d = sum(t.numel() * t.element_size() for t in hostin.values()) + off_h.numel() * 4
-        d2h = sum(t.numel() * t.element_size() for t in hostout.values())
+        d2h = sum(t.numel() * t.element_size() for t in hostout[0].values())
+        s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of a slot landed
+        ev_run = [torch.cuda.Event() for _ in range(2)]    # kernels of a slot done
+        ev_out = [torch.cuda.Event() for _ in range(2)]    # results of a slot copied out
+        for e in ev_run + ev_out:
+            e.record(s_run)
 
-        def e2e_step():
-            for n in dbuf:
-                dbuf[n].copy_(hostin[n], non_blocking=True)
-            doff.copy_(off_h, non_blocking=True)
-            binding.kmip_attn_fwd(dbuf["Q"], dbuf["K"], dbuf["V"], doff, N, H, d, k, scale,
-                                  out, idx, lse, stream)
-            binding.kmip_attn_bwd(dbuf["dO"], dbuf["Q"], dbuf["K"], dbuf["V"], idx, lse, dQ, dK,
-                                  dV, stream, N, H, d, k, scale)
-            for n, t in (("out", out), ("idx", idx), ("lse", lse), ("dQ", dQ), ("dK", dK),
-                         ("dV", dV)):
-                hostout[n].copy_(t, non_blocking=True)
+        def e2e_step(i):
+            j = i % 2
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_run[j])          # slot j's inputs no longer read
+                for n in dIn[j]:
+                    dIn[j][n].copy_(hostin[n], non_blocking=True)
+                dOff[j].copy_(off_h, non_blocking=True)
+                ev_in[j].record(s_in)
+            s_run.wait_event(ev_in[j])
+            s_run.wait_event(ev_out[j])             # slot j's results copied out
+            o = dOut[j]
+            rc = binding.kmip_attn_fwd(dIn[j]["Q"], dIn[j]["K"], dIn[j]["V"], dOff[j], N, H, d,
+                                       k, scale, o["out"], o["idx"], o["lse"], s_run)
+            if rc:
+                raise binding.KmipError(rc, "kmip_attn_fwd")
+            rc = binding.kmip_attn_bwd(dIn[j]["dO"], dIn[j]["Q"], dIn[j]["K"], dIn[j]["V"],
+                                       o["idx"], o["lse"], o["dQ"], o["dK"], o["dV"], s_run,
+                                       N, H, d, k, scale)
+            if rc:
+                raise binding.KmipError(rc, "kmip_attn_bwd")
+            ev_run[j].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_run[j])
+                for n, t in o.items():
+                    hostout[j][n].copy_(t, non_blocking=True)
+                ev_out[j].record(s_out)
 
-        for _ in range(args.warmup):
-            e2e_step()
+        for i in range(args.warmup):
+            e2e_step(i)
         torch.cuda.synchronize()
         if ws > 1:
             torch.distributed.barrier()
         e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e_a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e_b.record(stream)
+        e_a.record(s_in)
+        s_run.wait_event(e_a)
+        s_out.wait_event(e_a)
+        for i in range(args.steps):
+            e2e_step(i)
+        s_out.wait_event(ev_run[(args.steps - 1) % 2])
+        e_b.record(s_out)
         torch.cuda.synchronize()
         t_e2e = max_over_ranks([e_a.elapsed_time(e_b)], ws, dev)[0]
         binding.check_status()
+        last = hostout[(args.steps - 1) % 2]
+        if not torch.equal(last["idx"], idx.cpu()):
+            raise RuntimeError("end-to-end results differ from the device-resident run")
         e2e = {"value": job_throughput(N * H, ws, t_e2e / args.steps), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": t_e2e / args.steps}
+               "ms_per_step": t_e2e / args.steps, "streams": "copy-in, kernels, copy-out"}
 
     cpu = None
     if rank == 0 and ws == 1 and args.cpu_baseline:
