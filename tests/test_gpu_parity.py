@@ -89,6 +89,15 @@ def test_small_shapes(dev, dtype, d, k):
     _full_compare(inp, res, k, scale)
 
 
+@pytest.mark.parametrize("d,k", [(32, 15), (128, 16), (16, 64), (64, 45)])
+def test_max_heads(dev, d, k):
+    # 64 heads: rows of H * d * 2 bytes (up to 16 KiB) in the tensor maps and
+    # 64 work items per graph slice.
+    inp = wl.random_case([300, 5, 171], H=64, d=d, dtype="bf16", seed=900 + d + k)
+    res = _run(dev, inp, k, 1.0 / np.sqrt(d))
+    _full_compare(inp, res, k, 1.0 / np.sqrt(d))
+
+
 def test_single_graph_null_offsets(dev):
     inp = wl.random_case([777], H=3, d=32, dtype="bf16", seed=4)
     a = _run(dev, inp, 15, 0.2, bwd=False, use_offsets=True)
