@@ -160,9 +160,11 @@ kmip_status_t kmip_get_status(kmip_stream_t stream);
 
 /*
  * Which forward kernel kmip_attn_fwd runs for these sizes: 1 = the tcgen05
- * tensor-core kernel (bf16 inputs whose top-k lists, queues and K ring fit
- * in shared memory), 0 = the fp32-FMA kernel, -1 = unsupported arguments.
- * Pure host logic; touches no device.
+ * tensor-core kernel (bf16 inputs whose top-k lists, record buffers, Q tiles
+ * and two K stages fit in shared memory: d = 16 or 32 with any k <= 64,
+ * d = 64 with k <= 48, d = 128 with k <= 16), 0 = the fp32-FMA kernel (fp32
+ * inputs and the other bf16 shapes), -1 = unsupported arguments.  Pure host
+ * logic; touches no device.
  */
 int kmip_fwd_path(int d, int k, kmip_dtype_t dtype);
 
