@@ -430,8 +430,9 @@ def run_reference(args, ws, rank):
 
 
 def run_profile_calls(args):
-    """A few forward calls of the workload and nothing else: the command an
-    ncu capture of the forward kernel runs (no timing loop, no baselines)."""
+    """A few forward calls of the workload and nothing else (with --profile-bwd:
+    one forward, then that many backward calls): the command an ncu capture of
+    one kernel runs (no timing loop, no baselines)."""
     import dataclasses
     w = wl.WORKLOADS[args.workload]
     if args.nodes:
@@ -440,13 +441,19 @@ def run_profile_calls(args):
         w = dataclasses.replace(w, N=args.nodes)
     k = args.k or w.k
     dev = torch.device("cuda", 0)
-    inp = wl.make_inputs(w, with_grad_out=False)
+    inp = wl.make_inputs(w, with_grad_out=args.profile_bwd)
     g = {n: t.to(dev) for n, t in inp.items()}
-    for _ in range(args.profile_calls):
-        binding.attn_fwd(g["Q"], g["K"], g["V"], k, w.scale, g["offsets"])
+    if args.profile_bwd:
+        out, idx, lse = binding.attn_fwd(g["Q"], g["K"], g["V"], k, w.scale, g["offsets"])
+        for _ in range(args.profile_calls):
+            binding.attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, w.scale)
+    else:
+        for _ in range(args.profile_calls):
+            binding.attn_fwd(g["Q"], g["K"], g["V"], k, w.scale, g["offsets"])
     torch.cuda.synchronize()
     binding.check_status()
-    print(json.dumps({"profile_calls": args.profile_calls, "workload": w.name, "N": w.N, "k": k}))
+    print(json.dumps({"profile_calls": args.profile_calls, "workload": w.name, "N": w.N, "k": k,
+                      "kernel": "bwd" if args.profile_bwd else "fwd"}))
 
 
 def main():
@@ -465,6 +472,8 @@ def main():
                     help="override N of a single-graph workload (profiling only)")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="run this many forward calls and exit (for ncu captures)")
+    ap.add_argument("--profile-bwd", action="store_true",
+                    help="with --profile-calls: one forward, then backward calls")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
