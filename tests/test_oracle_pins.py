@@ -34,7 +34,8 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "handworked.json")
 def _ev(expr) -> float:
     if isinstance(expr, (int, float)):
         return float(expr)
-    return float(eval(expr, {"__builtins__": {}}, {"ln": math.log, "Fraction": Fraction}))
+    return float(eval(expr, {"__builtins__": {}},
+                      {"ln": math.log, "Fraction": Fraction, "inf": math.inf}))
 
 
 def _arr(rows):
@@ -59,6 +60,11 @@ def test_golden_handworked(case):
     np.testing.assert_array_equal(r["idx"].reshape(N, k), np.array(case["idx"]))
     np.testing.assert_allclose(r["lse"].reshape(N), _arr(case["lse"]), rtol=0, atol=1e-13)
     np.testing.assert_allclose(r["out"].reshape(N, d), _arr(case["out"]), rtol=0, atol=1e-13)
+    # order statistics behind the parity rule: s_(k_eff), s_(k) - s_(k+1), decided
+    np.testing.assert_array_equal(r["kth"].reshape(N), _arr(case["kth"]))
+    np.testing.assert_array_equal(r["gap"].reshape(N), _arr(case["gap"]))
+    np.testing.assert_array_equal(oracle.decided(r["gap"], r["kth"]).reshape(N),
+                                  np.array(case["decided"]))
     if "dO" in case:
         dO = np.array(case["dO"], dtype=np.float64).reshape(N, H, d)
         g = oracle.given_idx(Q, K, V, r["idx"], off, scale, dO=dO)
@@ -148,6 +154,13 @@ def test_selection_brute_force_subsets(seed):
                 best = max(itertools.combinations(keys, keff), key=lambda S: sum(sc[j] for j in S))
                 assert set(r["idx"][i, h, :keff].tolist()) == set(best)
                 assert (r["idx"][i, h, keff:] == -1).all()
+                # order statistics by brute force: the smallest score of the
+                # best subset, and the best score outside it
+                kth = min(sc[j] for j in best)
+                rest = [sc[j] for j in keys if j not in best]
+                gap = kth - max(rest) if len(keys) > k else np.inf
+                assert abs(r["kth"][i, h] - kth) <= 1e-12
+                assert r["gap"][i, h] == gap if np.isinf(gap) else abs(r["gap"][i, h] - gap) <= 1e-12
 
 
 def test_selection_matches_torch_topk():

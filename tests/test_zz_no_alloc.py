@@ -3,17 +3,20 @@
 It exists for callers that cannot let the library allocate device memory
 (their own pool holds the GPU, their device has no stream-ordered pools, or
 they must not allocate once running).  It must give the same results as
-kmip_attn_fwd.  Two calls in a row with different inputs also show that the
-fixed work-list array, which keeps the previous call's contents, is fully
-rewritten by each call.
+kmip_attn_fwd, and -- checked on its own, so that a fault shared by both
+entry points cannot hide -- the same results as the fp64 oracle under the
+parity rules of tests/parity.py.  Two calls in a row with different inputs
+also show that the fixed work-list array, which keeps the previous call's
+contents, is fully rewritten by each call.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from graph_transformer_sparse_kmip_b200 import binding
 from graph_transformer_sparse_kmip_b200 import workloads as wl
-from parity import TOL, normwise
+from parity import TOL, check_selection, check_values, normwise
 
 pytestmark = pytest.mark.gpu
 
@@ -54,6 +57,13 @@ def test_noalloc_forward_matches_allocating_forward():
         assert torch.equal(i1, i2)
         assert normwise(o2.double().cpu().numpy(), o1.double().cpu().numpy()) <= tol
         assert normwise(l2.double().cpu().numpy(), l1.double().cpu().numpy()) <= tol
+        # and against the oracle, on the no-allocation call's own outputs
+        dt = inp["Q"].dtype
+        ref = oracle.fwd(inp["Q"], inp["K"], inp["V"], inp["offsets"], k, scale)
+        check_selection(inp["Q"], inp["K"], inp["offsets"], i2, ref)
+        given = oracle.given_idx(inp["Q"], inp["K"], inp["V"], i2.cpu(), inp["offsets"], scale)
+        check_values("out", o2, given["out"], dt)
+        check_values("lse", l2, given["lse"], dt)
 
 
 def test_noalloc_rejects_work_lists_beyond_its_array():
