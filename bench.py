@@ -170,97 +170,210 @@ def _flush(buf):
     buf.add_(1)  # read + write 256 MiB: evicts the 126 MB L2
 
 
+class SmClock:
+    """Instantaneous SM clock through NVML (None when NVML is unavailable)."""
+
+    def __init__(self, device: torch.device):
+        self.h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nv = pynvml
+        except Exception:
+            self.h = None
+
+    def read(self):
+        if self.h is None:
+            return None
+        try:
+            return int(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        except Exception:
+            return None
+
+
+def _bwd_bytes_per_unit(d: int, k: int, elem: int) -> int:
+    """Algorithmic bytes of the backward per (query, head): dO, Q rows
+    (elem * d each), lse (4), idx (4k), the k kept K and V rows
+    (2 k elem d), dQ (4d) and the fp32 dK/dV reductions (2 k 4 d, read and
+    written by the reduction unit: counted once each)."""
+    return 2 * elem * d + 4 + 4 * k + 2 * k * elem * d + 4 * d + 2 * k * 4 * d
+
+
+def _gather_bytes_per_unit(d: int, k: int, elem: int) -> int:
+    """Algorithmic bytes of the softmax + V gather per (query, head): the k
+    kept V rows, idx and out written, lse written."""
+    return k * (elem * d + 4) + elem * d + 4
+
+
+class Case:
+    """One workload's device inputs and output buffers."""
+
+    def __init__(self, w, k, dev, rank=0, nodes=None):
+        self.w, self.k = w, k
+        self.inp = rank_inputs(w, rank) if nodes is None else None
+        inp = self.inp
+        N, H, d = inp["Q"].shape
+        self.N, self.H, self.d = N, H, d
+        self.bwd = "bwd" in w.phases
+        self.g = {n: t.to(dev) for n, t in inp.items()}
+        self.out = torch.empty_like(self.g["Q"])
+        self.idx = torch.empty((N, H, k), dtype=torch.int32, device=dev)
+        self.lse = torch.empty((N, H), dtype=torch.float32, device=dev)
+        if self.bwd:
+            self.dQ = torch.empty((N, H, d), dtype=torch.float32, device=dev)
+            self.dK = torch.empty_like(self.dQ)
+            self.dV = torch.empty_like(self.dQ)
+        self.flops = _score_flops(inp["offsets"], H, d)
+        self.elem = self.g["Q"].element_size()
+
+    def fwd(self, stream, k=None, idx=None):
+        k = k or self.k
+        idx = self.idx if idx is None else idx
+        g = self.g
+        rc = binding.kmip_attn_fwd(g["Q"], g["K"], g["V"], g["offsets"], self.N, self.H, self.d,
+                                   k, self.w.scale, self.out, idx, self.lse, stream)
+        if rc:
+            raise binding.KmipError(rc, "kmip_attn_fwd")
+
+    def bwd_call(self, stream, k=None, idx=None):
+        k = k or self.k
+        idx = self.idx if idx is None else idx
+        g = self.g
+        rc = binding.kmip_attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, self.lse, self.dQ,
+                                   self.dK, self.dV, stream, self.N, self.H, self.d, k,
+                                   self.w.scale)
+        if rc:
+            raise binding.KmipError(rc, "kmip_attn_bwd")
+
+
+def time_case(case, stream, steps, warmup, flush, clock=None, k=None, idx=None):
+    """Per-step device times (ms) of the forward and the backward, each
+    bracketed by CUDA events on the launching stream, the L2 flushed
+    between steps outside the events; the SM clock read after every step."""
+    fwd_ms, bwd_ms, mhz = [], [], []
+    for it in range(warmup + steps):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        case.fwd(stream, k, idx)
+        e1.record(stream)
+        if case.bwd:
+            case.bwd_call(stream, k, idx)
+        e2.record(stream)
+        _flush(flush)
+        torch.cuda.synchronize()
+        if it >= warmup:
+            fwd_ms.append(e0.elapsed_time(e1))
+            bwd_ms.append(e1.elapsed_time(e2))
+            mhz.append(clock.read() if clock else None)
+    return fwd_ms, bwd_ms, mhz
+
+
+def _fp32_fma_peak_tflops(sms: int, mhz: float) -> float:
+    """fp32 FMA peak of the fp32-input forward: 128 FMA lanes per SM per
+    clock, 2 flops each."""
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def config_summary(case, fwd_ms, bwd_ms, peaks, sms, max_mhz):
+    N, H = case.N, case.H
+    f = statistics.mean(fwd_ms)
+    b = statistics.mean(bwd_ms)
+    path = binding.kmip_fwd_path(case.d, case.k, binding.dtype_code(case.g["Q"].dtype))
+    if path == 1:
+        peak, bound = float(peaks["bf16_tflops"]), "tensor (bf16, burst peak)"
+    else:
+        peak, bound = _fp32_fma_peak_tflops(sms, max_mhz or 1965.0), "fp32 fma (derived peak)"
+    ach = case.flops / (f * 1e-3) / 1e12
+    r = {"N": N, "H": H, "d": case.d, "k": case.k, "graphs": int(case.g["offsets"].numel() - 1),
+         "dtype": case.w.dtype, "steps": len(fwd_ms),
+         "fwd": {"ms": f, "ms_min": min(fwd_ms), "ms_max": max(fwd_ms),
+                 "query_heads_per_s": N * H / (f * 1e-3),
+                 "score_tflops": ach, "peak_tflops": peak, "frac": ach / peak, "bound": bound,
+                 "path": {1: "tcgen05 tensor cores", 0: "fp32 FMA"}.get(path, "?")}}
+    if case.bwd:
+        byts = N * H * _bwd_bytes_per_unit(case.d, case.k, case.elem)
+        r["bwd"] = {"ms": b, "algorithmic_bytes": byts, "gbs": byts / (b * 1e-3) / 1e9,
+                    "frac_hbm": byts / (b * 1e-3) / 1e9 / float(peaks["hbm_gbs"])}
+        r["fwd_bwd_query_heads_per_s"] = N * H / ((f + b) * 1e-3)
+    return r
+
+
 def run_ours(args, ws, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     binding.load()
     w = wl.WORKLOADS[args.workload]
     k = args.k or w.k
-    inp = rank_inputs(w, rank)
-    N, H, d = inp["Q"].shape
+    case = Case(w, k, dev, rank)
+    N, H, d = case.N, case.H, case.d
+    inp, g = case.inp, case.g
     scale = w.scale
-    g = {n: t.to(dev) for n, t in inp.items()}
     stream = torch.cuda.current_stream()
-    out = torch.empty_like(g["Q"])
-    idx = torch.empty((N, H, k), dtype=torch.int32, device=dev)
-    lse = torch.empty((N, H), dtype=torch.float32, device=dev)
-    dQ = torch.empty((N, H, d), dtype=torch.float32, device=dev)
-    dK = torch.empty_like(dQ)
-    dV = torch.empty_like(dQ)
     flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    clock = SmClock(dev)
 
-    def step():
-        rc = binding.kmip_attn_fwd(g["Q"], g["K"], g["V"], g["offsets"], N, H, d, k, scale,
-                                   out, idx, lse, stream)
-        if rc:
-            raise binding.KmipError(rc, "kmip_attn_fwd")
-        ev_mid.record(stream)
-        rc = binding.kmip_attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, dQ, dK, dV,
-                                   stream, N, H, d, k, scale)
-        if rc:
-            raise binding.KmipError(rc, "kmip_attn_bwd")
-
-    ev_mid = torch.cuda.Event(enable_timing=True)
     for _ in range(args.warmup):
-        step()
+        case.fwd(stream)
+        case.bwd_call(stream)
         _flush(flush)
     torch.cuda.synchronize()
     binding.check_status()
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
-        for s in range(args.steps):
-            a, m, b = evs[s]
-            a.record(stream)
-            ev_mid = m
-            step()
-            b.record(stream)
-            _flush(flush)
+        fwd_ms, bwd_ms, mhz = time_case(case, stream, args.steps, 0, flush, clock)
         torch.cuda.synchronize()
         if ws > 1:
             torch.distributed.barrier()
     binding.check_status()
-    fwd_ms = [a.elapsed_time(m) for a, m, _ in evs]
-    tot_ms = [a.elapsed_time(b) for a, _, b in evs]
-    t_fwd, t_tot = max_over_ranks([sum(fwd_ms), sum(tot_ms)], ws, dev)
+    tot_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)]
+    t_fwd, t_bwd, t_tot = max_over_ranks([sum(fwd_ms), sum(bwd_ms), sum(tot_ms)], ws, dev)
     ms_step = t_tot / args.steps
     ms_fwd = t_fwd / args.steps
+    ms_bwd = t_bwd / args.steps
     value = job_throughput(N * H, ws, ms_step)
     fwd_value = job_throughput(N * H, ws, ms_fwd)
+    idx_ref = case.idx.cpu()
 
     peaks, peak_kind = _peaks()
-    flops = _score_flops(inp["offsets"], H, d)
+    flops = case.flops
     achieved = flops / (ms_fwd * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
+    bwd_bytes = N * H * _bwd_bytes_per_unit(d, k, case.elem)
+    clocks = clk.summary()
 
-    # k sweep (rank 0 view; fwd+bwd ms per step, same timing rules, fewer steps)
+    # k sweep: forward and backward at the workload's other k values
     sweep = {}
     if args.k_sweep and w.k_sweep:
+        nsw = max(3, args.steps // 4)
         for ks in w.k_sweep:
             if ks == k:
-                sweep[str(ks)] = {"ms_fwd": round(ms_fwd, 4), "ms_fwd_bwd": round(ms_step, 4)}
+                sweep[str(ks)] = {"ms_fwd": ms_fwd, "ms_bwd": ms_bwd,
+                                  "frac": achieved / peak}
                 continue
             idx_s = torch.empty((N, H, ks), dtype=torch.int32, device=dev)
-            times = []
-            for it in range(args.warmup + max(3, args.steps // 2)):
-                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-                e0.record(stream)
-                binding.kmip_attn_fwd(g["Q"], g["K"], g["V"], g["offsets"], N, H, d, ks, scale,
-                                      out, idx_s, lse, stream)
-                e1.record(stream)
-                binding.kmip_attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx_s, lse, dQ, dK, dV,
-                                      stream, N, H, d, ks, scale)
-                e2.record(stream)
-                _flush(flush)
-                torch.cuda.synchronize()
-                if it >= args.warmup:
-                    times.append((e0.elapsed_time(e1), e0.elapsed_time(e2)))
-            sweep[str(ks)] = {"ms_fwd": round(statistics.mean(t[0] for t in times), 4),
-                              "ms_fwd_bwd": round(statistics.mean(t[1] for t in times), 4)}
+            f_ms, b_ms, _ = time_case(case, stream, nsw, 3, flush, None, ks, idx_s)
+            fm = statistics.mean(f_ms)
+            sweep[str(ks)] = {"ms_fwd": fm, "ms_bwd": statistics.mean(b_ms),
+                              "frac": flops / (fm * 1e-3) / 1e12 / peak}
+        binding.check_status()
+
+    # the other workloads: forward (and backward where the workload has one)
+    configs = {}
+    if args.configs and rank == 0:
+        for name, wo in wl.WORKLOADS.items():
+            if name == w.name:
+                continue
+            c2 = Case(wo, wo.k, dev)
+            f_ms, b_ms, _ = time_case(c2, stream, max(3, args.steps // 4), 3, flush)
+            configs[name] = config_summary(c2, f_ms, b_ms, peaks, sms, clocks.get("sm_max_mhz"))
+            del c2
         binding.check_status()
 
     # end to end through the public API: pinned host inputs in, host results out.
@@ -272,12 +385,13 @@ def run_ours(args, ws, rank, local):
     if args.e2e:
         hostin = {n: inp[n].pin_memory() for n in ("Q", "K", "V", "dO")}
         off_h = inp["offsets"].pin_memory()
-        outs = {"out": out, "idx": idx, "lse": lse, "dQ": dQ, "dK": dK, "dV": dV}
-        hostout = [{n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in outs.items()}
+        names = {"out": case.out, "idx": case.idx, "lse": case.lse, "dQ": case.dQ,
+                 "dK": case.dK, "dV": case.dV}
+        hostout = [{n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in names.items()}
                    for _ in range(2)]
         dIn = [{n: torch.empty_like(g[n]) for n in ("Q", "K", "V", "dO")} for _ in range(2)]
         dOff = [torch.empty_like(g["offsets"]) for _ in range(2)]
-        dOut = [outs, {n: torch.empty_like(t) for n, t in outs.items()}]
+        dOut = [{n: torch.empty_like(t) for n, t in names.items()} for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in hostin.values()) + off_h.numel() * 4
         d2h = sum(t.numel() * t.element_size() for t in hostout[0].values())
         s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
@@ -331,7 +445,7 @@ def run_ours(args, ws, rank, local):
         t_e2e = max_over_ranks([e_a.elapsed_time(e_b)], ws, dev)[0]
         binding.check_status()
         last = hostout[(args.steps - 1) % 2]
-        if not torch.equal(last["idx"], idx.cpu()):
+        if not torch.equal(last["idx"], idx_ref):
             raise RuntimeError("end-to-end results differ from the device-resident run")
         e2e = {"value": job_throughput(N * H, ws, t_e2e / args.steps), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -345,10 +459,10 @@ def run_ours(args, ws, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "N": N, "H": H, "d": d, "k": k, "graphs": int(
-            inp["offsets"].numel() - 1), "keys": w.values, "step": "fwd+bwd",
-            "parallelism": f"independent batch per GPU x{ws}",
-            "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "config": {"workload": w.name, "N": N, "H": H, "d": d, "k": k,
+                   "graphs": int(inp["offsets"].numel() - 1), "keys": w.values,
+                   "step": "fwd+bwd", "parallelism": f"independent batch per GPU x{ws}",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
         "fwd": {"value": fwd_value, "unit": UNIT, "ms_per_step": ms_fwd},
         "roofline": {"bound": "tensor", "kernel": "forward (score + top-k + softmax + gather)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -357,15 +471,28 @@ def run_ours(args, ws, rank, local):
                      "algorithmic_flops_per_launch": flops,
                      "path": {1: "tcgen05 tensor cores", 0: "fp32 FMA"}.get(
                          binding.kmip_fwd_path(d, k, binding.dtype_code(g["Q"].dtype)), "?")},
+        "phases": {
+            "fwd": {"ms": ms_fwd, "score_tflops": achieved, "frac_bf16_peak": achieved / peak,
+                    "gather_bytes_per_launch": N * H * _gather_bytes_per_unit(d, k, case.elem)},
+            "bwd": {"ms": ms_bwd, "algorithmic_bytes": bwd_bytes,
+                    "gbs": bwd_bytes / (ms_bwd * 1e-3) / 1e9,
+                    "frac_hbm": bwd_bytes / (ms_bwd * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                    "hbm_peak_gbs": float(peaks["hbm_gbs"]), "peak_source": peak_kind},
+        },
+        "per_step": {"ms_fwd": [round(x, 4) for x in fwd_ms],
+                     "ms_bwd": [round(x, 4) for x in bwd_ms],
+                     "sm_mhz_after_step": mhz},
         "gpu_launches": 3 * args.steps,
     }
     if sweep:
         res["k_sweep"] = sweep
+    if configs:
+        res["configs"] = configs
     if e2e:
         res["e2e"] = e2e
     if cpu:
         res["cpu_baseline"] = cpu
-    res["clocks"] = clk.summary()
+    res["clocks"] = clocks
     return res
 
 
@@ -395,12 +522,16 @@ def cpu_baseline(inp, k, scale, budget_s=15.0, pairs_per_batch=None):
         done += len(pq)
         batch += 1
     return {"value": done / t_used, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "pairs": done,
             "sample": f"{done} (query, head) pairs of the same workload in {batch} batches; "
                       f"fwd (all-key fp64 scores + full sort) and bwd; {t_used:.1f} s"}
 
 
 def run_reference(args, ws, rank):
-    """The oracle as the reference arm: bounded sample per step, host cores."""
+    """The oracle as the reference arm: each step is a bounded sample of
+    (query, head) pairs of the same workload on the host cores.  value is
+    the sampled pairs per second; ms_per_step is the real wall time of one
+    sampled step (the full-step time it would take is reported apart)."""
     if rank != 0:
         return None
     w = wl.WORKLOADS[args.workload]
@@ -408,21 +539,29 @@ def run_reference(args, ws, rank):
     inp = wl.make_inputs(w, with_grad_out=True)
     N, H = inp["Q"].shape[:2]
     per_step_s = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
-    vals, samples = [], []
+    vals, samples, walls = [], [], []
     for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         r = cpu_baseline(inp, k, w.scale, budget_s=per_step_s)
+        wall = time.perf_counter() - t0
         if s >= args.warmup:
             vals.append(r["value"])
             samples.append(r)
+            walls.append(wall)
     value = statistics.mean(vals)
-    ms_step = N * H / value * 1e3
+    pairs = [r["pairs"] for r in samples]
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(walls) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "N": N, "H": H, "d": w.d, "k": k, "step": "fwd+bwd",
-                   "parallelism": "host cores (oracle)"},
+        "config": {"workload": w.name, "N": N, "H": H, "d": w.d, "k": k,
+                   "graphs": int(inp["offsets"].numel() - 1), "keys": w.values,
+                   "step": "fwd+bwd", "parallelism": "host cores (oracle)",
+                   "l2": "not applicable (host)"},
+        "sample_pairs_per_step": statistics.mean(pairs),
+        "full_step_ms_extrapolated": N * H / value * 1e3,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[-1]["cores"],
                          "kind": "oracle", "sample": samples[-1]["sample"] + " per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -467,6 +606,8 @@ def main():
     ap.add_argument("--no-k-sweep", dest="k_sweep", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip timing the other workloads")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--nodes", type=int, default=None,
                     help="override N of a single-graph workload (profiling only)")
@@ -478,6 +619,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = _dist()
+    if args.gpus != ws:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {ws}: launch N > 1 ranks with "
+                 "torchrun (one process per GPU)")
     if args.profile_calls:
         run_profile_calls(args)
         return

@@ -3,10 +3,10 @@
  * graph transformers on NVIDIA B200 (sm_100a).
  *
  * The operation (k-Maximum Inner Product Attention for Graph Transformers
- * and the Expressive Power of GraphGPS, Abstract: "selects the most relevant
- * key nodes per query via a top-k operation", combined with a score
- * computation whose memory is linear in the node count): for query node i
- * of graph g and head h,
+ * and the Expressive Power of GraphGPS, Abstract: each query attends only to
+ * the keys whose inner product with it is among the k largest, and the
+ * scores are computed without ever storing them all, so memory grows
+ * linearly with the node count): for query node i of graph g and head h,
  *
  *   s_j  = Q[i,h,:] . K[j,h,:]          for every node j of graph g
  *   S    = the k_eff = min(k, n_g) keys with the largest s_j
@@ -29,9 +29,10 @@
  *
  * Memory: the N x N score matrix is never materialised; scores live in
  * tensor memory / registers only.  The library's own device memory is a
- * work list of O(H * (N / 128 + G)) 16-byte items per forward call, taken
- * from the stream-ordered allocator of the current device and released on
- * the same stream.
+ * work list of O(N / q + G) 16-byte items per forward call (q = 256 queries
+ * per item on the tensor-core path, 128 otherwise; the same items serve
+ * every head), taken from the stream-ordered allocator of the current
+ * device and released on the same stream.
  *
  * Conventions common to every call:
  *   - All tensor pointers are DEVICE pointers on the current CUDA device
