@@ -51,6 +51,9 @@ def _load():
         lib.kmip_oracle_given_idx.argtypes = [P, P, P, P, P, P, I64, I64, I32, I32, I32,
                                               F64, P, P, P, P, P]
         lib.kmip_oracle_given_idx.restype = I32
+        lib.kmip_oracle_full.argtypes = [P, P, P, P, I64, I64, I32, I32, F64, P, P, I64, P, P,
+                                         I32]
+        lib.kmip_oracle_full.restype = I32
         _lib = lib
     return _lib
 
@@ -145,6 +148,30 @@ def given_idx(Q, K, V, idx, offsets, scale: float, dO=None):
     if rc:
         raise ValueError(f"kmip_oracle_given_idx failed with code {rc}")
     return res
+
+
+def full_attention(Q, K, V, offsets, scale: float, pairs_q=None, pairs_h=None,
+                   nthreads: int | None = None):
+    """Full softmax attention over every key of each query's graph (the
+    comparison of Figure 8).  Returns dict(out, lse): [N, H, d] / [N, H] for
+    every pair, or [n, d] / [n] for the listed pairs."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    N, H, d = Q.shape
+    off = _offsets(offsets, N)
+    if pairs_q is None:
+        out = np.zeros((N, H, d)); lse = np.zeros((N, H)); pq = ph = None; n = 0
+    else:
+        pq = np.ascontiguousarray(pairs_q, dtype=np.int64)
+        ph = np.ascontiguousarray(pairs_h, dtype=np.int32)
+        n = len(pq)
+        out = np.zeros((n, d)); lse = np.zeros(n)
+    rc = _load().kmip_oracle_full(_p(Q), _p(K), _p(V), _p(off), len(off) - 1, N, H, d,
+                                  float(scale), None if pq is None else _p(pq),
+                                  None if ph is None else _p(ph), n, _p(out), _p(lse),
+                                  nthreads or default_threads())
+    if rc:
+        raise ValueError(f"kmip_oracle_full failed with code {rc}")
+    return dict(out=out, lse=lse)
 
 
 def decided(gap: np.ndarray, kth: np.ndarray, rel: float = 1e-3) -> np.ndarray:

@@ -310,3 +310,109 @@ int kmip_oracle_given_idx(const double* Q, const double* K, const double* V,
   free(s); free(p); free(dp);
   return rc;
 }
+
+/*
+ * Full softmax attention over every key of the query's graph, for the
+ * diagnostics that compare k-MIP attention with it (k-Maximum Inner Product
+ * Attention for Graph Transformers ..., Figure 8: the L2 distance between
+ * the two outputs, and the share of the full softmax weight that the k kept
+ * keys carry).  For query i of graph g and head h:
+ *
+ *   lse_full = log sum_{j in g} exp(scale * s_j)     (max-shifted)
+ *   out_full = sum_{j in g} exp(scale * s_j - lse_full) V[j,h,:]
+ *
+ * For a list of (query, head) pairs (pairs_q == NULL: every pair, rows in
+ * (i, h) order).  Returns 0, or 1 on malformed offsets, 2 on a bad pair.
+ */
+typedef struct {
+  const double *Q, *K, *V;
+  const int64_t* offsets;
+  int64_t G, N;
+  int H, d;
+  double scale;
+  const int64_t* pairs_q;
+  const int32_t* pairs_h;
+  int64_t npairs;
+  double* out;
+  double* lse;
+  int64_t next;
+  pthread_mutex_t lock;
+} full_ctx;
+
+static void full_one(const full_ctx* c, int64_t i, int h, int64_t row, double* s) {
+  const int d = c->d, H = c->H;
+  int64_t g = graph_of(c->offsets, c->G, i);
+  int64_t j0 = c->offsets[g], j1 = c->offsets[g + 1];
+  const double* q = c->Q + (i * H + h) * (int64_t)d;
+  double m = -INFINITY;
+  for (int64_t j = j0; j < j1; ++j) {
+    const double* kr = c->K + (j * H + h) * (int64_t)d;
+    double acc = 0.0;
+    for (int t = 0; t < d; ++t) acc += q[t] * kr[t];
+    s[j - j0] = c->scale * acc;
+    if (s[j - j0] > m) m = s[j - j0];
+  }
+  double sum = 0.0;
+  for (int64_t j = j0; j < j1; ++j) sum += exp(s[j - j0] - m);
+  double L = m + log(sum);
+  c->lse[row] = L;
+  double* o = c->out + row * (int64_t)d;
+  for (int t = 0; t < d; ++t) o[t] = 0.0;
+  for (int64_t j = j0; j < j1; ++j) {
+    double p = exp(s[j - j0] - L);
+    const double* vr = c->V + (j * H + h) * (int64_t)d;
+    for (int t = 0; t < d; ++t) o[t] += p * vr[t];
+  }
+}
+
+static void* full_worker(void* arg) {
+  full_ctx* c = (full_ctx*)arg;
+  int64_t maxn = 1;
+  for (int64_t g = 0; g < c->G; ++g)
+    if (c->offsets[g + 1] - c->offsets[g] > maxn) maxn = c->offsets[g + 1] - c->offsets[g];
+  double* s = (double*)malloc(sizeof(double) * (size_t)maxn);
+  if (!s) return (void*)1;
+  int64_t total = c->pairs_q ? c->npairs : c->N * c->H;
+  for (;;) {
+    pthread_mutex_lock(&c->lock);
+    int64_t t = c->next;
+    c->next += 16;
+    pthread_mutex_unlock(&c->lock);
+    if (t >= total) break;
+    int64_t e = t + 16 < total ? t + 16 : total;
+    for (; t < e; ++t) {
+      if (c->pairs_q) full_one(c, c->pairs_q[t], c->pairs_h[t], t, s);
+      else full_one(c, t / c->H, (int)(t % c->H), t, s);
+    }
+  }
+  free(s);
+  return NULL;
+}
+
+int kmip_oracle_full(const double* Q, const double* K, const double* V,
+                     const int64_t* offsets, int64_t G, int64_t N, int H, int d,
+                     double scale, const int64_t* pairs_q, const int32_t* pairs_h,
+                     int64_t npairs, double* out, double* lse, int nthreads) {
+  if (check_offsets(offsets, G, N)) return 1;
+  if (pairs_q)
+    for (int64_t t = 0; t < npairs; ++t)
+      if (pairs_q[t] < 0 || pairs_q[t] >= N || pairs_h[t] < 0 || pairs_h[t] >= H) return 2;
+  full_ctx c;
+  memset(&c, 0, sizeof c);
+  c.Q = Q; c.K = K; c.V = V; c.offsets = offsets; c.G = G; c.N = N; c.H = H; c.d = d;
+  c.scale = scale; c.pairs_q = pairs_q; c.pairs_h = pairs_h; c.npairs = npairs;
+  c.out = out; c.lse = lse;
+  if (nthreads < 1) nthreads = 1;
+  pthread_mutex_init(&c.lock, NULL);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  int rc = 0;
+  for (int t = 0; t < nthreads; ++t) pthread_create(&th[t], NULL, full_worker, &c);
+  for (int t = 0; t < nthreads; ++t) {
+    void* r = NULL;
+    pthread_join(th[t], &r);
+    if (r) rc = 3;
+  }
+  free(th);
+  pthread_mutex_destroy(&c.lock);
+  return rc;
+}

@@ -306,3 +306,36 @@ def test_workload_generators_are_seeded():
     sizes = np.diff(a["offsets"].numpy())
     assert len(sizes) == 64 and sizes.min() >= 300 and sizes.max() <= 600
     assert a["Q"].dtype == torch.bfloat16 and a["Q"].shape == (int(sizes.sum()), 4, 32)
+
+
+# --- full softmax attention (the comparison of Figure 8) ---
+
+@pytest.mark.parametrize("seed", [0, 3])
+def test_full_attention_matches_torch_dense(seed):
+    sizes = [6, 11, 0, 4]
+    c = wl.random_case(sizes, H=2, d=5, dtype="f32", seed=seed, with_grad_out=False)
+    Q, K, V = (c[n].double().numpy() for n in ("Q", "K", "V"))
+    off = c["offsets"].numpy().astype(np.int64)
+    r = oracle.full_attention(Q, K, V, off, 0.6, nthreads=2)
+    _, _, _, out, lse = _dense_attention_fp64(Q, K, V, off, 0.6)
+    np.testing.assert_allclose(r["out"], out.detach().numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], lse.detach().numpy(), rtol=0, atol=1e-12)
+    pq = np.array([0, 7, 20]); ph = np.array([1, 0, 1], dtype=np.int32)
+    rp = oracle.full_attention(Q, K, V, off, 0.6, pq, ph)
+    np.testing.assert_array_equal(rp["out"], r["out"][pq, ph])
+
+
+def test_topk_weight_share_rises_to_one():
+    """exp(lse_k - lse_full) is the softmax weight the k kept keys carry:
+    it grows with k and reaches 1 once k covers the graph."""
+    c = wl.random_case([40], H=1, d=8, dtype="f32", seed=2, with_grad_out=False)
+    Q, K, V = (c[n].double().numpy() for n in ("Q", "K", "V"))
+    full = oracle.full_attention(Q, K, V, None, 0.5)
+    prev = np.zeros(40)
+    for k in (1, 3, 10, 39, 40, 45):
+        r = oracle.fwd(Q, K, V, None, k, 0.5)
+        share = np.exp(r["lse"] - full["lse"]).reshape(-1)
+        assert (share <= 1 + 1e-12).all() and (share >= prev - 1e-12).all()
+        prev = share
+    np.testing.assert_allclose(prev, 1.0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["out"], full["out"], rtol=0, atol=1e-12)
