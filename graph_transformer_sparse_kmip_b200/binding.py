@@ -19,8 +19,9 @@ KMIP_BF16, KMIP_F32 = 0, 1
 STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTED",
                 3: "KMIP_ERR_CUDA", 4: "KMIP_ERR_BAD_OFFSETS", 5: "KMIP_ERR_TIMEOUT",
                 6: "KMIP_ERR_BAD_INDEX", 7: "KMIP_ERR_SCRATCH_LIMIT"}
-EXPORTED = ("kmip_attn_fwd", "kmip_attn_fwd_noalloc", "kmip_attn_bwd", "kmip_get_status",
-            "kmip_error_string", "kmip_fwd_path", "kmip_version")
+EXPORTED = ("kmip_attn_fwd", "kmip_attn_fwd_noalloc", "kmip_attn_fwd_diag", "kmip_attn_bwd",
+            "kmip_attn_bwd_deterministic", "kmip_get_status", "kmip_error_string",
+            "kmip_fwd_path", "kmip_version")
 
 _lib = None
 
@@ -45,8 +46,13 @@ def load() -> ctypes.CDLL:
     lib.kmip_attn_fwd.restype = I32
     lib.kmip_attn_fwd_noalloc.argtypes = lib.kmip_attn_fwd.argtypes
     lib.kmip_attn_fwd_noalloc.restype = I32
+    lib.kmip_attn_fwd_diag.argtypes = [P, P, P, P, I64, I32, I32, I32, F32, P, P, P, P, P, I32,
+                                       I32]
+    lib.kmip_attn_fwd_diag.restype = I32
     lib.kmip_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, F32, I32]
     lib.kmip_attn_bwd.restype = I32
+    lib.kmip_attn_bwd_deterministic.argtypes = lib.kmip_attn_bwd.argtypes
+    lib.kmip_attn_bwd_deterministic.restype = I32
     lib.kmip_get_status.argtypes = [P]
     lib.kmip_get_status.restype = I32
     lib.kmip_error_string.argtypes = [I32]
@@ -118,6 +124,22 @@ def kmip_attn_fwd_noalloc(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, l
                                         int(dtype))
 
 
+def kmip_attn_fwd_diag(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, lse_all,
+                       stream=None, num_graphs=None, dtype=None) -> int:
+    """kmip_attn_fwd plus lse_all [N, H]: the log-sum-exp over every key of
+    the query's graph (the normaliser of full softmax attention)."""
+    _check_cuda(Q, K, V, graph_offsets, out, idx, lse, lse_all)
+    G = (graph_offsets.numel() - 1) if graph_offsets is not None else 1
+    if num_graphs is None:
+        num_graphs = G
+    if dtype is None:
+        dtype = dtype_code(Q.dtype)
+    return load().kmip_attn_fwd_diag(_ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N),
+                                     int(H), int(d), int(k), float(scale), _ptr(out), _ptr(idx),
+                                     _ptr(lse), _ptr(lse_all), _stream(stream), int(num_graphs),
+                                     int(dtype))
+
+
 def kmip_attn_bwd(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None, N=None, H=None, d=None,
                   k=None, scale=None, dtype=None) -> int:
     _check_cuda(dOut, Q, K, V, idx, lse, dQ, dK, dV)
@@ -131,6 +153,23 @@ def kmip_attn_bwd(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None, N=None, H=No
     return load().kmip_attn_bwd(_ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse),
                                 _ptr(dQ), _ptr(dK), _ptr(dV), _stream(stream), int(N), int(H),
                                 int(d), int(k), float(scale), int(dtype))
+
+
+def kmip_attn_bwd_deterministic(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None, N=None,
+                                H=None, d=None, k=None, scale=None, dtype=None) -> int:
+    """kmip_attn_bwd with bitwise reproducible dK/dV (sorted gather, no
+    atomics)."""
+    _check_cuda(dOut, Q, K, V, idx, lse, dQ, dK, dV)
+    N_, H_, d_ = Q.shape
+    N = N_ if N is None else N
+    H = H_ if H is None else H
+    d = d_ if d is None else d
+    k = idx.shape[-1] if k is None else k
+    if dtype is None:
+        dtype = dtype_code(Q.dtype)
+    return load().kmip_attn_bwd_deterministic(
+        _ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse), _ptr(dQ), _ptr(dK),
+        _ptr(dV), _stream(stream), int(N), int(H), int(d), int(k), float(scale), int(dtype))
 
 
 def kmip_get_status(stream=None) -> int:
@@ -169,14 +208,30 @@ def attn_fwd(Q, K, V, k: int, scale: float, graph_offsets=None, stream=None):
     return out, idx, lse
 
 
-def attn_bwd(dOut, Q, K, V, idx, lse, scale: float, stream=None):
+def attn_fwd_diag(Q, K, V, k: int, scale: float, graph_offsets=None, stream=None):
+    """Returns (out, idx, lse, lse_all): kmip_attn_fwd's outputs and the
+    log-sum-exp over every key of the query's graph."""
+    N, H, d = Q.shape
+    out = torch.empty_like(Q)
+    idx = torch.empty((N, H, k), dtype=torch.int32, device=Q.device)
+    lse = torch.empty((N, H), dtype=torch.float32, device=Q.device)
+    lse_all = torch.empty((N, H), dtype=torch.float32, device=Q.device)
+    rc = kmip_attn_fwd_diag(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, lse_all,
+                            stream)
+    if rc:
+        raise KmipError(rc, "kmip_attn_fwd_diag")
+    return out, idx, lse, lse_all
+
+
+def attn_bwd(dOut, Q, K, V, idx, lse, scale: float, stream=None, deterministic=False):
     """Returns (dQ, dK, dV), fp32 [N,H,d]."""
     dQ = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
     dK = torch.empty_like(dQ)
     dV = torch.empty_like(dQ)
-    rc = kmip_attn_bwd(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream, scale=scale)
+    fn = kmip_attn_bwd_deterministic if deterministic else kmip_attn_bwd
+    rc = fn(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream, scale=scale)
     if rc:
-        raise KmipError(rc, "kmip_attn_bwd")
+        raise KmipError(rc, fn.__name__)
     return dQ, dK, dV
 
 

@@ -75,11 +75,14 @@ int device_sm_count() {
 
 using namespace kmip;
 
-KMIP_EXPORT kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void* V,
-                                        const int32_t* graph_offsets, int64_t N, int H, int d,
-                                        int k, float scale, void* out, int32_t* idx, float* lse,
-                                        kmip_stream_t stream_, int num_graphs,
-                                        kmip_dtype_t dtype) {
+namespace {
+
+// The forward of kmip_attn_fwd and kmip_attn_fwd_diag (lse_all = nullptr:
+// no all-key diagnostics).
+kmip_status_t attn_fwd_impl(const void* Q, const void* K, const void* V,
+                            const int32_t* graph_offsets, int64_t N, int H, int d, int k,
+                            float scale, void* out, int32_t* idx, float* lse, float* lse_all,
+                            kmip_stream_t stream_, int num_graphs, kmip_dtype_t dtype) {
   kmip_status_t st = check_common(N, H, d, k, scale, dtype);
   if (st != KMIP_OK) return st;
   if (graph_offsets && num_graphs < 1) return KMIP_ERR_INVALID_ARG;
@@ -110,7 +113,8 @@ KMIP_EXPORT kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void
   cudaError_t e = launch_worklist(graph_offsets, G, (int)N, qpi, items, count, (int)max_items,
                                   status, stream);
   if (e == cudaSuccess) {
-    FwdArgs a{Q, K, V, (int)N, H, d, k, scale, out, idx, lse, items, count, (int)max_items, status};
+    FwdArgs a{Q, K, V, (int)N, H, d, k, scale, out, idx, lse, items, count, (int)max_items, status,
+              lse_all};
     e = tc ? launch_fwd_tc(a, stream) : launch_fwd_simt(dtype, a, stream);
   }
   cudaError_t ef = cudaFreeAsync(scratch, stream);
@@ -121,11 +125,33 @@ KMIP_EXPORT kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void
   return KMIP_OK;
 }
 
-KMIP_EXPORT kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K,
-                                        const void* V, const int32_t* idx, const float* lse,
-                                        float* dQ, float* dK, float* dV, kmip_stream_t stream_,
-                                        int64_t N, int H, int d, int k, float scale,
+}  // namespace
+
+KMIP_EXPORT kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void* V,
+                                        const int32_t* graph_offsets, int64_t N, int H, int d,
+                                        int k, float scale, void* out, int32_t* idx, float* lse,
+                                        kmip_stream_t stream, int num_graphs,
                                         kmip_dtype_t dtype) {
+  return attn_fwd_impl(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, nullptr,
+                       stream, num_graphs, dtype);
+}
+
+KMIP_EXPORT kmip_status_t kmip_attn_fwd_diag(const void* Q, const void* K, const void* V,
+                                             const int32_t* graph_offsets, int64_t N, int H,
+                                             int d, int k, float scale, void* out, int32_t* idx,
+                                             float* lse, float* lse_all, kmip_stream_t stream,
+                                             int num_graphs, kmip_dtype_t dtype) {
+  if (N > 0 && !lse_all) return KMIP_ERR_INVALID_ARG;
+  return attn_fwd_impl(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, lse_all,
+                       stream, num_graphs, dtype);
+}
+
+namespace {
+
+kmip_status_t attn_bwd_impl(const void* dOut, const void* Q, const void* K, const void* V,
+                            const int32_t* idx, const float* lse, float* dQ, float* dK,
+                            float* dV, kmip_stream_t stream_, int64_t N, int H, int d, int k,
+                            float scale, kmip_dtype_t dtype, bool deterministic) {
   kmip_status_t st = check_common(N, H, d, k, scale, dtype);
   if (st != KMIP_OK) return st;
   if (N == 0) return KMIP_OK;
@@ -136,18 +162,47 @@ KMIP_EXPORT kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const v
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   int* status = status_ptr();
   if (!status) return KMIP_ERR_CUDA;
-  const size_t bytes = sizeof(float) * (size_t)N * H * d;
-  cudaError_t e = cudaMemsetAsync(dK, 0, bytes, stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, bytes, stream);
-  if (e == cudaSuccess) {
-    BwdArgs a{dOut, Q, K, V, idx, lse, dQ, dK, dV, (int)N, H, d, k, scale, status};
-    e = launch_bwd(dtype, a, stream);
+  BwdArgs a{dOut, Q, K, V, idx, lse, dQ, dK, dV, (int)N, H, d, k, scale, status};
+  cudaError_t e;
+  if (deterministic) {
+    e = launch_bwd_deterministic(dtype, a, stream);
+    if (e == cudaErrorNotSupported) {
+      cudaGetLastError();
+      return KMIP_ERR_UNSUPPORTED;
+    }
+  } else {
+    const size_t bytes = sizeof(float) * (size_t)N * H * d;
+    e = cudaMemsetAsync(dK, 0, bytes, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dV, 0, bytes, stream);
+    if (e == cudaSuccess) e = launch_bwd(dtype, a, stream);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
     return KMIP_ERR_CUDA;
   }
   return KMIP_OK;
+}
+
+}  // namespace
+
+KMIP_EXPORT kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K,
+                                        const void* V, const int32_t* idx, const float* lse,
+                                        float* dQ, float* dK, float* dV, kmip_stream_t stream,
+                                        int64_t N, int H, int d, int k, float scale,
+                                        kmip_dtype_t dtype) {
+  return attn_bwd_impl(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream, N, H, d, k, scale, dtype,
+                       false);
+}
+
+KMIP_EXPORT kmip_status_t kmip_attn_bwd_deterministic(const void* dOut, const void* Q,
+                                                      const void* K, const void* V,
+                                                      const int32_t* idx, const float* lse,
+                                                      float* dQ, float* dK, float* dV,
+                                                      kmip_stream_t stream, int64_t N, int H,
+                                                      int d, int k, float scale,
+                                                      kmip_dtype_t dtype) {
+  return attn_bwd_impl(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream, N, H, d, k, scale, dtype,
+                       true);
 }
 
 KMIP_EXPORT kmip_status_t kmip_get_status(kmip_stream_t stream_) {

@@ -38,12 +38,12 @@ __device__ __forceinline__ void topk_insert(float* ls, int* li, int& cnt, int k,
   if (cnt == k) thr = ls[(k - 1) * kThreads + x];
 }
 
-template <typename T, int D, int KCAP>
+template <typename T, int D, int KCAP, bool DIAG>
 __global__ void __launch_bounds__(kThreads)
 fwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
                 const WorkItem* __restrict__ items, const int* __restrict__ count_ptr, int H,
                 int k, float scale, T* __restrict__ out, int32_t* __restrict__ idx,
-                float* __restrict__ lse) {
+                float* __restrict__ lse, float* __restrict__ lse_all) {
   using VT = Vec<T>;
   constexpr int VN = VT::N;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -66,6 +66,9 @@ fwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __res
     }
     float thr = -INFINITY;
     int cnt = 0;
+    // all-key diagnostics: running maximum and sum of exp2(c2 (s - max))
+    const float c2 = scale * 1.4426950408889634f;
+    float dmax = -INFINITY, dsum = 0.f;
 
     for (int jt = it.j0; jt < it.j1; jt += kKeyTile) {
       const int nt = min(kKeyTile, it.j1 - jt);
@@ -102,6 +105,14 @@ fwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __res
           }
           const float s = a0 + a1;
           if (s > thr) topk_insert(ls, li, cnt, k, s, jt + r, thr);
+          if constexpr (DIAG) {
+            if (s > dmax) {
+              dsum = dsum * exp2f((dmax - s) * c2) + 1.f;
+              dmax = s;
+            } else {
+              dsum += exp2f((s - dmax) * c2);
+            }
+          }
         }
       }
     }
@@ -132,13 +143,14 @@ fwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __res
       for (int c = 0; c < D; c += VN) VT::store(out + row * D + c, o + c);
       for (int t = 0; t < k; ++t) idx[row * k + t] = t < cnt ? li[t * kThreads + x] : -1;
       lse[row] = L;
+      if constexpr (DIAG) lse_all[row] = (dmax * c2 + log2f(dsum)) * 0.6931471805599453f;
     }
   }
 }
 
-template <typename T, int D, int KCAP>
-cudaError_t launch_typed(const FwdArgs& a, cudaStream_t stream) {
-  auto kern = fwd_simt_kernel<T, D, KCAP>;
+template <typename T, int D, int KCAP, bool DIAG>
+cudaError_t launch_diag(const FwdArgs& a, cudaStream_t stream) {
+  auto kern = fwd_simt_kernel<T, D, KCAP, DIAG>;
   const size_t smem = sizeof(float) * (kKeyTile * D + 2 * KCAP * kThreads);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -146,8 +158,14 @@ cudaError_t launch_typed(const FwdArgs& a, cudaStream_t stream) {
   const int grid = (int)(blocks < 65535 * 16 ? blocks : 65535 * 16);
   kern<<<grid, kThreads, smem, stream>>>(
       static_cast<const T*>(a.Q), static_cast<const T*>(a.K), static_cast<const T*>(a.V), a.items,
-      a.count, a.H, a.k, a.scale, static_cast<T*>(a.out), a.idx, a.lse);
+      a.count, a.H, a.k, a.scale, static_cast<T*>(a.out), a.idx, a.lse, a.lse_all);
   return cudaGetLastError();
+}
+
+template <typename T, int D, int KCAP>
+cudaError_t launch_typed(const FwdArgs& a, cudaStream_t stream) {
+  if (a.lse_all) return launch_diag<T, D, KCAP, true>(a, stream);
+  return launch_diag<T, D, KCAP, false>(a, stream);
 }
 
 template <typename T, int D>

@@ -43,7 +43,8 @@
 //                 filters already work on the next item.
 // The warpgroups rebalance their registers at the start (setmaxnreg): the
 // producer/MMA warpgroup and the inserters give some up, and the filters,
-// which hold a tile's scores, take them.
+// which hold a tile's scores, take them (32 / 160 / 64 per thread: the split
+// the filters and inserters compile into without spilling scores).
 // Keys outside the query's graph are never loaded (the key range comes from
 // the work item); the last tile of a graph masks its tail columns.
 //
@@ -83,7 +84,7 @@ constexpr size_t kMinSmem = 120 * 1024;  // keeps one CTA (one TMEM owner) per S
 // Registers per thread: at launch, and after the warpgroups rebalance them
 // (producer/MMA warpgroup and inserters give some up, filters take them).
 constexpr int kLaunchRegs = 96;
-constexpr int kRegsCtl = 40, kRegsFilter = 152, kRegsInsert = 64;
+constexpr int kRegsCtl = 32, kRegsFilter = 160, kRegsInsert = 64;
 static_assert(kThreads % 128 == 0, "whole warpgroups");
 static_assert(128 * kRegsCtl + 32 * kFilterWarps * kRegsFilter + 32 * kInsertWarps * kRegsInsert <=
                   kThreads * kLaunchRegs,
@@ -150,6 +151,8 @@ struct Cfg {
 
 struct TcParams {
   const __nv_bfloat16* V;
+  float* lse_all;  // with the all-key diagnostics: log-sum-exp over every key
+  float c2;        // scale * log2(e)
   const WorkItem* items;
   const int* count;
   int H, k;
@@ -169,12 +172,14 @@ __device__ __forceinline__ float max16(const float* x) {
   return fmax3(fmax3(a, b, c), fmax3(d, e, x[15]), -INFINITY);
 }
 
-// A row's top-k list is its line of shared memory: scores ls[0 .. KCAP-1]
-// and keys li[...], larger score first, equal scores by smaller key.  For
-// KCAP == kRegK the list always has kRegK slots: the first kRegK - k hold
-// +inf sentinels, the k real entries follow, so the k-th best is always the
-// last slot; otherwise the k real entries are slots 0 .. k-1.  Unused slots
-// hold -inf and key -1.
+// A row's top-k list is its line of shared memory: scores ls[..] and keys
+// li[..].  For KCAP == kRegK it is a sorted list of kRegK slots, larger score
+// first: the first kRegK - k slots hold +inf sentinels and the k real entries
+// follow, so the k-th best is always the last slot.  For larger KCAP the k
+// entries form a binary heap with the worst entry at the root (slot 0):
+// entry a is worse than entry b when a's score is smaller, or equal with a
+// larger key; the root's score is the row's threshold.  Unused entries hold
+// -inf and key -1.
 template <int KCAP>
 __device__ __forceinline__ int first_slot(int k) {
   return KCAP == kRegK ? kRegK - k : 0;
@@ -193,6 +198,51 @@ __device__ __forceinline__ void list_reset(float* ls, int* li, int k) {
       ls[t] = -INFINITY;
       li[t] = -1;
     }
+  }
+}
+
+// (sa, ja) is worse than (sb, jb): smaller score, or equal score and larger
+// key.  Padding entries (-inf, -1) are worse than every real entry.
+__device__ __forceinline__ bool worse(float sa, int ja, float sb, int jb) {
+  return sa < sb || (sa == sb && ja > jb);
+}
+
+// Put (s, j) at slot `pos` of the heap of n entries and sift it down to
+// where both children are no worse than it.
+__device__ __forceinline__ void heap_sift(float* H, int* J, int n, int pos, float s, int j) {
+  for (;;) {
+    const int l = 2 * pos + 1;
+    if (l >= n) break;
+    int c = l;
+    float cs = H[l];
+    int cj = J[l];
+    if (l + 1 < n) {
+      const float rs = H[l + 1];
+      const int rj = J[l + 1];
+      if (worse(rs, rj, cs, cj)) {
+        c = l + 1;
+        cs = rs;
+        cj = rj;
+      }
+    }
+    if (!worse(cs, cj, s, j)) break;
+    H[pos] = cs;
+    J[pos] = cj;
+    pos = c;
+  }
+  H[pos] = s;
+  J[pos] = j;
+}
+
+// Heap of n entries -> sorted list, best first (heap sort: the worst entry
+// is moved to the back, then the next worst, ...).
+__device__ __forceinline__ void heap_to_sorted(float* H, int* J, int n) {
+  for (int end = n - 1; end > 0; --end) {
+    const float s = H[end];
+    const int j = J[end];
+    H[end] = H[0];
+    J[end] = J[0];
+    heap_sift(H, J, end, 0, s, j);
   }
 }
 
@@ -238,13 +288,16 @@ __device__ __forceinline__ bool next_candidate(uint64_t& m, const float* rs, con
 }
 
 // Insertion for k <= kRegK: the list is held in registers and every lane
-// takes one candidate per round through a branch-free compare-exchange
-// chain.  Records are visited in key order, so an equal score stays behind
-// the entries already listed.  Returns the new threshold.  Out of line so
-// that its code exists once.
+// takes one candidate per round.  A candidate beats the last slot (the k-th
+// best), so it replaces it and then moves up while it is strictly larger
+// than the entry before it; the rounds stop moving as soon as no lane's
+// candidate moves, which in the steady state (candidates just above the
+// threshold) is after a step or two.  Records are visited in key order, so
+// an equal score stays behind the entries already listed.  Returns the new
+// threshold.
 template <int NREC>
 __device__ __forceinline__ float insert_regs(float* ls, int* li, const float* rs, const int* rj,
-                                          int rn, float thr) {
+                                             int rn, float thr) {
   uint64_t m = record_bits<NREC>(rs, rn, thr);
   if (!__any_sync(0xffffffffu, m != 0)) return thr;
   float L[kRegK];
@@ -259,17 +312,20 @@ __device__ __forceinline__ float insert_regs(float* ls, int* li, const float* rs
     int j = -1;
     const bool have = next_candidate(m, rs, rj, thr, s, j);
     if (!__any_sync(0xffffffffu, have)) break;
-    // Compare-exchange chain: the larger value stays, the smaller moves on
-    // (a lane without a candidate passes -inf through, changing nothing).
+    if (have) {
+      L[kRegK - 1] = s;
+      J[kRegK - 1] = j;
+    }
 #pragma unroll
-    for (int t = 0; t < kRegK; ++t) {
-      const bool c = s > L[t];
-      const float hi = fmaxf(L[t], s), lo = fminf(L[t], s);
-      const int jk = c ? j : J[t], jm = c ? J[t] : j;
-      L[t] = hi;
-      s = lo;
-      J[t] = jk;
-      j = jm;
+    for (int t = kRegK - 1; t > 0; --t) {
+      const bool up = L[t] > L[t - 1];
+      if (!__any_sync(0xffffffffu, up)) break;
+      const float a = L[t], b = L[t - 1];
+      const int ja = J[t], jb = J[t - 1];
+      L[t - 1] = up ? a : b;
+      L[t] = up ? b : a;
+      J[t - 1] = up ? ja : jb;
+      J[t] = up ? jb : ja;
     }
     thr = L[kRegK - 1];
   }
@@ -282,36 +338,24 @@ __device__ __forceinline__ float insert_regs(float* ls, int* li, const float* rs
   return thr;
 }
 
-// Insertion for larger k: binary search and shift in shared memory over the
-// k real entries starting at slot `first`, one candidate after another in
-// key order (an equal score stays behind).  Returns the new threshold.
+// Insertion for larger k: every recorded score that still beats the root of
+// the row's heap replaces the root and sifts down (log k steps in shared
+// memory, whatever the candidate's rank).  Returns the new threshold.
 template <int NREC>
-__device__ __forceinline__ float insert_smem(float* ls, int* li, const float* rs, const int* rj,
-                                          int rn, float thr, int k, int first) {
+__device__ __forceinline__ float insert_heap(float* H, int* J, const float* rs, const int* rj,
+                                             int rn, float thr, int k) {
   uint64_t m = record_bits<NREC>(rs, rn, thr);
-  float* L = ls + first;
-  int* J = li + first;
   float s;
   int jn;
   while (next_candidate(m, rs, rj, thr, s, jn)) {
-    int lo = 0, hi = k - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (L[mid] < s) hi = mid; else lo = mid + 1;
-    }
-    for (int e = k - 1; e > lo; --e) {
-      L[e] = L[e - 1];
-      J[e] = J[e - 1];
-    }
-    L[lo] = s;
-    J[lo] = jn;
-    thr = L[k - 1];
+    heap_sift(H, J, k, 0, s, jn);
+    thr = H[0];
   }
   __syncwarp();
   return thr;
 }
 
-template <int D, int KCAP>
+template <int D, int KCAP, bool DIAG>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const TcParams p) {
@@ -540,6 +584,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const bool tile_on = mt == 0 || (it.q1 - it.q0) > kBM;  // warp-uniform
       ++item;
       thr = -INFINITY;
+      // all-key diagnostics: running maximum and sum of exp2(c2 (s - max))
+      float dmax = -INFINITY, dsum = 0.f;
       const int ntiles = (it.j1 - it.j0 + kBN - 1) / kBN;
       for (int t = 0; t < ntiles; ++t, ++tn) {
         const int b = (int)(tn % kNB);
@@ -580,11 +626,31 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             for (int u = 0; u < 32; ++u)
               if (c * 32 + u >= valid) v[c][u] = -INFINITY;
         }
-        uint32_t mask = 0;
+        float gm[kBN / 16];  // maxima of the eight 16-key groups
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) {
-          if (max16(v[c]) > thr) mask |= 1u << (2 * c);
-          if (max16(v[c] + 16) > thr) mask |= 1u << (2 * c + 1);
+          gm[2 * c] = max16(v[c]);
+          gm[2 * c + 1] = max16(v[c] + 16);
+        }
+        uint32_t mask = 0;
+#pragma unroll
+        for (int g = 0; g < kBN / 16; ++g) mask |= (gm[g] > thr ? 1u : 0u) << g;
+        if constexpr (DIAG) {
+          // Softmax normaliser over every key of the graph (online: the sum
+          // is rescaled whenever the running maximum rises).
+          const float tm = fmax3(fmax3(gm[0], gm[1], gm[2]), fmax3(gm[3], gm[4], gm[5]),
+                                 fmaxf(gm[6], gm[7]));
+          if (tm > dmax) {
+            dsum *= exp2f((dmax - tm) * p.c2);
+            dmax = tm;
+          }
+          if (dmax > -INFINITY) {
+            const float off = dmax * p.c2;
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c)
+#pragma unroll
+              for (int u = 0; u < 32; ++u) dsum += exp2f(fmaf(v[c][u], p.c2, -off));
+          }
         }
         const uint32_t todo = __reduce_or_sync(0xffffffffu, mask);
         if (todo) {
@@ -604,14 +670,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               }
             }
           }
+          // Hand a batch over early once enough rows hold records and the
+          // insert warp has nothing else queued.
+          if (ok && __popc(__ballot_sync(0xffffffffu, rn > 0)) >= kHandLanes && other_free())
+            hand_over(0);
         }
         if (!ok) break;
-        // Hand a batch over early once enough rows hold records and the
-        // insert warp has nothing else queued.
-        if (__popc(__ballot_sync(0xffffffffu, rn > 0)) >= kHandLanes && other_free())
-          hand_over(0);
       }
       if (!ok) break;
+      if constexpr (DIAG) {
+        const int i = it.q0 + mt * kBM + quarter * 32 + lane;
+        if (tile_on && i < it.q1)
+          p.lse_all[(int64_t)i * p.H + (int)(w / count)] = (dmax * p.c2 + log2f(dsum)) * 0.6931471805599453f;
+      }
       hand_over(1);  // the item's last batch
     }
   } else {
@@ -653,7 +724,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (KCAP == kRegK)
           thr = insert_regs<NR>(L, J, rs, rj, rn, thr);
         else
-          thr = insert_smem<NR>(L, J, rs, rj, rn, thr, p.k, first_slot<KCAP>(p.k));
+          thr = insert_heap<NR>(L, J, rs, rj, rn, thr, p.k);
         {
           // Publish the row's threshold with the item it belongs to, in one
           // 8-byte store, for the filter to raise its own.
@@ -668,6 +739,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       if (!ok) break;
       if (tile_on && i < it.q1) {
+        if (KCAP != kRegK) heap_to_sorted(L, J, p.k);
         const float* Lf = L + first_slot<KCAP>(p.k);
         const int* Jf = J + first_slot<KCAP>(p.k);
         int cnt = 0;
@@ -754,14 +826,14 @@ bool make_map(CUtensorMap* m, const void* ptr, int N, int H) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int KCAP>
+template <int D, int KCAP, bool DIAG>
 cudaError_t launch_cfg(const FwdArgs& a, cudaStream_t stream) {
   using C = Cfg<D, KCAP>;
   static_assert(C::kFits, "shared memory budget");
   CUtensorMap mq, mk;
   if (!make_map<D>(&mq, a.Q, a.N, a.H) || !make_map<D>(&mk, a.K, a.N, a.H))
     return cudaErrorInvalidValue;
-  auto kern = fwd_tc_kernel<D, KCAP>;
+  auto kern = fwd_tc_kernel<D, KCAP, DIAG>;
   // The warpgroups' register split draws on the launch allocation: refuse
   // to launch a build whose kernel was given fewer registers.
   cudaFuncAttributes fa;
@@ -773,7 +845,8 @@ cudaError_t launch_cfg(const FwdArgs& a, cudaStream_t stream) {
   const int64_t units = (int64_t)a.H * a.max_items;
   const int sms = device_sm_count();
   const int grid = (int)(units < sms ? units : sms);
-  TcParams p{static_cast<const __nv_bfloat16*>(a.V), a.items, a.count, a.H, a.k, a.scale,
+  TcParams p{static_cast<const __nv_bfloat16*>(a.V), a.lse_all, a.scale * 1.4426950408889634f,
+             a.items, a.count, a.H, a.k, a.scale,
              static_cast<__nv_bfloat16*>(a.out), a.idx, a.lse, a.status, kTimeoutNs};
   kern<<<grid, kThreads, C::kSmemLaunch, stream>>>(mq, mk, p);
   return cudaGetLastError();
@@ -781,7 +854,10 @@ cudaError_t launch_cfg(const FwdArgs& a, cudaStream_t stream) {
 
 template <int D, int KCAP>
 cudaError_t launch_k(const FwdArgs& a, cudaStream_t stream) {
-  if constexpr (Cfg<D, KCAP>::kFits) return launch_cfg<D, KCAP>(a, stream);
+  if constexpr (Cfg<D, KCAP>::kFits) {
+    if (a.lse_all) return launch_cfg<D, KCAP, true>(a, stream);
+    return launch_cfg<D, KCAP, false>(a, stream);
+  }
   return cudaErrorNotSupported;
 }
 

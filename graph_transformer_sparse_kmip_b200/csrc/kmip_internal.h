@@ -22,6 +22,19 @@ struct FwdArgs {
   const int* count;       // number of items (device)
   int max_items;          // host-side upper bound on *count
   int* status;            // device status word
+  float* lse_all = nullptr;  // [N, H] log-sum-exp over every key, or nullptr
+};
+
+// Buffers of the deterministic backward (all device, E = N H k entries):
+// per kept key its (p, scale dS) coefficients, its (key, head) bucket as a
+// sort key (sentinel for padding) and its position in idx; per bucket the
+// number of kept keys that point to it.
+struct DetBuffers {
+  float2* coef = nullptr;
+  uint32_t* keys = nullptr;
+  uint32_t* vals = nullptr;
+  int* count = nullptr;
+  uint32_t sentinel = 0;
 };
 
 struct BwdArgs {
@@ -37,6 +50,7 @@ struct BwdArgs {
   int N, H, d, k;
   float scale;
   int* status;
+  DetBuffers det = {};  // keys != nullptr: write coefficients instead of scattering
 };
 
 // Queries per work item of each forward kernel (the tensor-core forward
@@ -61,6 +75,11 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 bool fwd_tc_supported(int d, int k);
 
 cudaError_t launch_bwd(kmip_dtype_t dtype, const BwdArgs& a, cudaStream_t stream);
+
+// Deterministic backward: coefficients, a stable sort of the kept keys by
+// (key, head) and an in-order reduction per key (kmip_bwd_det.cu).  Takes
+// its scratch from the stream-ordered allocator.
+cudaError_t launch_bwd_deterministic(kmip_dtype_t dtype, const BwdArgs& a, cudaStream_t stream);
 
 int device_sm_count();
 

@@ -137,6 +137,26 @@ kmip_status_t kmip_attn_fwd_noalloc(const void* Q, const void* K, const void* V,
                                     kmip_stream_t stream, int num_graphs, kmip_dtype_t dtype);
 
 /*
+ * Forward pass with the all-key diagnostics (k-Maximum Inner Product
+ * Attention for Graph Transformers ..., Figure 8: how far k-MIP attention is
+ * from full softmax attention).  Same arguments and results as
+ * kmip_attn_fwd, plus
+ *   lse_all        [N, H] fp32 (device), overwritten: the log-sum-exp of the
+ *                  scaled scores over EVERY key of the query's graph, i.e.
+ *                  the normaliser of full softmax attention.
+ * exp(lse - lse_all) is the share of the full softmax weight that the k kept
+ * keys carry (1 when k covers the graph).  The scores are the same ones the
+ * selection uses; the sum is accumulated in fp32 with one exp2 per score, so
+ * this call is slower than kmip_attn_fwd.  lse_all may not be NULL when
+ * N > 0 (KMIP_ERR_INVALID_ARG).
+ */
+kmip_status_t kmip_attn_fwd_diag(const void* Q, const void* K, const void* V,
+                                 const int32_t* graph_offsets, int64_t N, int H, int d, int k,
+                                 float scale, void* out, int32_t* idx, float* lse,
+                                 float* lse_all, kmip_stream_t stream, int num_graphs,
+                                 kmip_dtype_t dtype);
+
+/*
  * Backward pass.
  *   dOut           [N, H, d] of `dtype` (device): gradient of the loss w.r.t. out.
  *   Q, K, V        the forward's inputs; idx, lse the forward's outputs.
@@ -151,6 +171,24 @@ kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K, cons
                             const int32_t* idx, const float* lse, float* dQ, float* dK,
                             float* dV, kmip_stream_t stream, int64_t N, int H, int d, int k,
                             float scale, kmip_dtype_t dtype);
+
+/*
+ * Backward pass with bitwise reproducible gradients.  Same arguments and
+ * results as kmip_attn_bwd, computed without atomic additions: the kept keys
+ * are sorted by (key, head) with a stable radix sort, and each key's dK and
+ * dV rows are summed by one warp over its queries in the order of their
+ * positions in idx, so repeated calls on the same inputs return identical
+ * bits.  Takes O(N H k) scratch (about 28 bytes per kept key plus 4 per
+ * (node, head)) from the stream-ordered allocator of the current device and
+ * releases it on the same stream.  Returns KMIP_ERR_UNSUPPORTED when
+ * N H k >= 2^32 - 1 or the sort's scans would exceed 2^24 entries
+ * (N H k > about 2.7e8); otherwise as kmip_attn_bwd.
+ */
+kmip_status_t kmip_attn_bwd_deterministic(const void* dOut, const void* Q, const void* K,
+                                          const void* V, const int32_t* idx, const float* lse,
+                                          float* dQ, float* dK, float* dV, kmip_stream_t stream,
+                                          int64_t N, int H, int d, int k, float scale,
+                                          kmip_dtype_t dtype);
 
 /*
  * Synchronises `stream`, then returns and clears the current device's status

@@ -203,3 +203,112 @@ def test_gmm_n100000(dev, k):
 
 def test_pointcloud_n524288(dev):
     _large(dev, "pointcloud_n524288", n_pairs=128)
+
+
+# --- all-key diagnostics (kmip_attn_fwd_diag) ---
+
+def _diag_compare(dev, inp, k, scale, pairs=None):
+    g = _to(dev, inp)
+    out, idx, lse, lse_all = binding.attn_fwd_diag(g["Q"], g["K"], g["V"], k, scale, g["offsets"])
+    torch.cuda.synchronize()
+    binding.check_status()
+    # same selection and outputs as the plain forward
+    o2, i2, l2 = binding.attn_fwd(g["Q"], g["K"], g["V"], k, scale, g["offsets"])
+    assert torch.equal(idx, i2) and torch.equal(out, o2) and torch.equal(lse, l2)
+    dt = inp["Q"].dtype
+    if pairs is None:
+        full = oracle.full_attention(inp["Q"], inp["K"], inp["V"], inp["offsets"], scale)
+        check_values("lse_all", lse_all, full["lse"], dt)
+        got = lse_all.cpu().double().numpy()
+    else:
+        pq, ph = pairs
+        full = oracle.full_attention(inp["Q"], inp["K"], inp["V"], inp["offsets"], scale, pq, ph)
+        got = lse_all.cpu().double().numpy()[pq, ph]
+        check_values("lse_all(sample)", got, full["lse"], dt)
+    # the kept keys' share of the full softmax weight lies in (0, 1]
+    share = np.exp(lse.cpu().double().numpy() - lse_all.cpu().double().numpy())
+    assert (share > 0).all() and (share <= 1 + 2 * TOL[dt]).all()
+    return share
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d,k", [(16, 5), (32, 15), (64, 45), (128, 16)])
+def test_diag_lse_all_small(dev, dtype, d, k):
+    inp = wl.random_case(SIZES, H=2, d=d, dtype=dtype, seed=7 * d + k)
+    _diag_compare(dev, inp, k, 1.0 / np.sqrt(d))
+
+
+def test_diag_k_covering_the_graph_is_full_attention(dev):
+    inp = wl.random_case([30, 5, 0, 64], H=2, d=32, dtype="bf16", seed=5)
+    share = _diag_compare(dev, inp, 64, 0.2)
+    np.testing.assert_allclose(share, 1.0, rtol=0, atol=1e-4)
+
+
+def test_diag_graph_n31623(dev):
+    w = wl.WORKLOADS["graph_n31623"]
+    inp = wl.make_inputs(w, with_grad_out=False)
+    N, H = inp["Q"].shape[:2]
+    pq, ph = wl.sample_pairs(N, H, 256, seed=3)
+    _diag_compare(dev, inp, w.k, w.scale, (pq.numpy(), ph.numpy()))
+
+
+# --- deterministic backward (kmip_attn_bwd_deterministic) ---
+
+def _det_compare(dev, inp, k, scale):
+    g = _to(dev, inp)
+    out, idx, lse = binding.attn_fwd(g["Q"], g["K"], g["V"], k, scale, g["offsets"])
+    a = binding.attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, scale, deterministic=True)
+    b = binding.attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, scale, deterministic=True)
+    atomic = binding.attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, scale)
+    torch.cuda.synchronize()
+    binding.check_status()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y), "deterministic backward differs between two runs"
+    assert torch.equal(a[0], atomic[0])  # dQ is the same computation in both
+    dt = inp["Q"].dtype
+    given = oracle.given_idx(inp["Q"], inp["K"], inp["V"], idx.cpu(), inp["offsets"], scale,
+                             dO=inp["dO"])
+    for name, x in zip(("dQ", "dK", "dV"), a):
+        check_values(name, x, given[name], dt)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d,k", [(16, 64), (32, 15), (64, 45), (128, 5)])
+def test_deterministic_bwd_small(dev, dtype, d, k):
+    inp = wl.random_case(SIZES, H=2, d=d, dtype=dtype, seed=3 * d + k)
+    _det_compare(dev, inp, k, 1.0 / np.sqrt(d))
+
+
+def test_deterministic_bwd_gmm_n100000(dev):
+    w = wl.WORKLOADS["gmm_n100000"]
+    _det_compare(dev, wl.make_inputs(w), w.k, w.scale)
+
+
+# --- exact ties: the smaller key index wins ---
+
+@pytest.mark.parametrize("dtype,d,k", [("bf16", 32, 15), ("bf16", 16, 45), ("f32", 32, 15),
+                                       ("bf16", 64, 5)])
+def test_exact_ties_go_to_the_smaller_index(dev, dtype, d, k):
+    """Many keys are exact copies of one strong key, so their scores tie
+    bit for bit (the same products summed in the same order) and the k-th and
+    (k+1)-th best are equal.  The pages give no tie rule; the library's (and
+    the oracle's) is larger score first, then the smaller node index, so on
+    every exactly tied pair the kept set must be the oracle's."""
+    sizes = [700, 300]
+    inp = wl.random_case(sizes, H=2, d=d, dtype=dtype, seed=77 + d)
+    K = inp["K"].clone()
+    for h in range(2):
+        strong = K[5, h] * 3                      # one key far above the rest
+        for j in list(range(100, 160)) + list(range(720, 740)):
+            K[j, h] = strong
+        K[650, h] = strong
+    inp["K"] = K
+    res = _run(dev, inp, k, 1.0 / np.sqrt(d), bwd=False)
+    ref = oracle.fwd(inp["Q"], inp["K"], inp["V"], inp["offsets"], k, 1.0 / np.sqrt(d))
+    got = res["idx"].cpu().numpy()
+    # where the oracle's k-th and (k+1)-th scores tie exactly, the kept set
+    # must still be the oracle's (ties to the smaller index)
+    tied = ref["gap"] == 0
+    assert tied.sum() > 100
+    same = (np.sort(got, -1) == np.sort(ref["idx"], -1)).all(-1)
+    assert same[tied].all(), f"{(~same[tied]).sum()} tied pairs keep other keys"
