@@ -13,7 +13,12 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libkmip.so")
+# KMIP_DEBUG_BOUNDS=1 loads the build with device-side index checks
+# (python -m graph_transformer_sparse_kmip_b200.build --debug-bounds).
+LIB_PATH = os.path.join(_PKG, "libkmip_debug.so" if os.environ.get("KMIP_DEBUG_BOUNDS") == "1"
+                        else "libkmip.so")
+# KMIP_NVTX=1 wraps every library call in an NVTX range (for nsys/ncu timelines).
+_NVTX = os.environ.get("KMIP_NVTX") == "1"
 
 KMIP_BF16, KMIP_F32 = 0, 1
 STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTED",
@@ -71,6 +76,18 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _call(name, *args):
+    """Calls the C entry point `name` (inside an NVTX range when KMIP_NVTX=1)."""
+    fn = getattr(load(), name)
+    if not _NVTX:
+        return fn(*args)
+    torch.cuda.nvtx.range_push(name)
+    try:
+        return fn(*args)
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -101,7 +118,7 @@ def kmip_attn_fwd(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse, stre
         num_graphs = G
     if dtype is None:
         dtype = dtype_code(Q.dtype)
-    return load().kmip_attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N), int(H),
+    return _call("kmip_attn_fwd", _ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N), int(H),
                                 int(d), int(k), float(scale), _ptr(out), _ptr(idx), _ptr(lse),
                                 _stream(stream), int(num_graphs), int(dtype))
 
@@ -118,7 +135,7 @@ def kmip_attn_fwd_noalloc(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, l
         num_graphs = G
     if dtype is None:
         dtype = dtype_code(Q.dtype)
-    return load().kmip_attn_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N),
+    return _call("kmip_attn_fwd_noalloc", _ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N),
                                         int(H), int(d), int(k), float(scale), _ptr(out),
                                         _ptr(idx), _ptr(lse), _stream(stream), int(num_graphs),
                                         int(dtype))
@@ -134,7 +151,7 @@ def kmip_attn_fwd_diag(Q, K, V, graph_offsets, N, H, d, k, scale, out, idx, lse,
         num_graphs = G
     if dtype is None:
         dtype = dtype_code(Q.dtype)
-    return load().kmip_attn_fwd_diag(_ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N),
+    return _call("kmip_attn_fwd_diag", _ptr(Q), _ptr(K), _ptr(V), _ptr(graph_offsets), int(N),
                                      int(H), int(d), int(k), float(scale), _ptr(out), _ptr(idx),
                                      _ptr(lse), _ptr(lse_all), _stream(stream), int(num_graphs),
                                      int(dtype))
@@ -150,7 +167,7 @@ def kmip_attn_bwd(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None, N=None, H=No
     k = idx.shape[-1] if k is None else k
     if dtype is None:
         dtype = dtype_code(Q.dtype)
-    return load().kmip_attn_bwd(_ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse),
+    return _call("kmip_attn_bwd", _ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse),
                                 _ptr(dQ), _ptr(dK), _ptr(dV), _stream(stream), int(N), int(H),
                                 int(d), int(k), float(scale), int(dtype))
 
@@ -167,8 +184,8 @@ def kmip_attn_bwd_deterministic(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None
     k = idx.shape[-1] if k is None else k
     if dtype is None:
         dtype = dtype_code(Q.dtype)
-    return load().kmip_attn_bwd_deterministic(
-        _ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse), _ptr(dQ), _ptr(dK),
+    return _call(
+        "kmip_attn_bwd_deterministic", _ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse), _ptr(dQ), _ptr(dK),
         _ptr(dV), _stream(stream), int(N), int(H), int(d), int(k), float(scale), int(dtype))
 
 
