@@ -348,6 +348,43 @@ def run_ours(args, ws, rank, local):
     bwd_bytes = N * H * _bwd_bytes_per_unit(d, k, case.elem)
     clocks = clk.summary()
 
+    # the softmax + V gather stage by itself (kmip_attn_gather over the
+    # forward's sets): what the fused forward's last stage moves, plus the
+    # K rows it needs to recompute the kept scores
+    gat_ms = []
+    o_g, l_g = torch.empty_like(case.out), torch.empty_like(case.lse)
+    for it in range(3 + max(3, args.steps // 2)):
+        _flush(flush)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        rc = binding.kmip_attn_gather(g["Q"], g["K"], g["V"], case.idx, N, H, d, k, scale, o_g,
+                                      l_g, stream)
+        b_.record(stream)
+        if rc:
+            raise binding.KmipError(rc, "kmip_attn_gather")
+        torch.cuda.synchronize()
+        if it >= 3:
+            gat_ms.append(a_.elapsed_time(b_))
+    gat_ms_mean = statistics.mean(gat_ms)
+    # the deterministic backward (sorted gather, no atomics) on the same step
+    det_ms = []
+    for it in range(3 + max(3, args.steps // 2)):
+        _flush(flush)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        rc = binding.kmip_attn_bwd_deterministic(g["dO"], g["Q"], g["K"], g["V"], case.idx,
+                                                 case.lse, case.dQ, case.dK, case.dV, stream,
+                                                 N, H, d, k, scale)
+        b_.record(stream)
+        if rc:
+            raise binding.KmipError(rc, "kmip_attn_bwd_deterministic")
+        torch.cuda.synchronize()
+        if it >= 3:
+            det_ms.append(a_.elapsed_time(b_))
+    binding.check_status()
+    gat_bytes = N * H * (_gather_bytes_per_unit(d, k, case.elem) + k * case.elem * d + case.elem * d)
+    del o_g, l_g
+
     # k sweep: forward and backward at the workload's other k values
     sweep = {}
     if args.k_sweep and w.k_sweep:
@@ -478,6 +515,12 @@ def run_ours(args, ws, rank, local):
         "phases": {
             "fwd": {"ms": ms_fwd, "score_tflops": achieved, "frac_bf16_peak": achieved / peak,
                     "gather_bytes_per_launch": N * H * _gather_bytes_per_unit(d, k, case.elem)},
+            "gather_stage": {"kernel": "kmip_attn_gather (softmax + V gather over the forward's sets)",
+                             "ms": gat_ms_mean, "algorithmic_bytes": gat_bytes,
+                             "gbs": gat_bytes / (gat_ms_mean * 1e-3) / 1e9,
+                             "frac_hbm": gat_bytes / (gat_ms_mean * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
+            "bwd_deterministic": {"ms": statistics.mean(det_ms),
+                                  "kernels": "coefficients + stable radix sort + in-order gather"},
             "bwd": {"ms": ms_bwd, "algorithmic_bytes": bwd_bytes,
                     "gbs": bwd_bytes / (ms_bwd * 1e-3) / 1e9,
                     "frac_hbm": bwd_bytes / (ms_bwd * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),

@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTE
                 3: "KMIP_ERR_CUDA", 4: "KMIP_ERR_BAD_OFFSETS", 5: "KMIP_ERR_TIMEOUT",
                 6: "KMIP_ERR_BAD_INDEX", 7: "KMIP_ERR_SCRATCH_LIMIT"}
 EXPORTED = ("kmip_attn_fwd", "kmip_attn_fwd_noalloc", "kmip_attn_fwd_diag", "kmip_attn_bwd",
-            "kmip_attn_bwd_deterministic", "kmip_get_status", "kmip_error_string",
+            "kmip_attn_bwd_deterministic", "kmip_attn_gather", "kmip_get_status",
+            "kmip_error_string",
             "kmip_fwd_path", "kmip_version")
 
 _lib = None
@@ -58,6 +59,8 @@ def load() -> ctypes.CDLL:
     lib.kmip_attn_bwd.restype = I32
     lib.kmip_attn_bwd_deterministic.argtypes = lib.kmip_attn_bwd.argtypes
     lib.kmip_attn_bwd_deterministic.restype = I32
+    lib.kmip_attn_gather.argtypes = [P, P, P, P, I64, I32, I32, I32, F32, P, P, P, I32]
+    lib.kmip_attn_gather.restype = I32
     lib.kmip_get_status.argtypes = [P]
     lib.kmip_get_status.restype = I32
     lib.kmip_error_string.argtypes = [I32]
@@ -187,6 +190,26 @@ def kmip_attn_bwd_deterministic(dOut, Q, K, V, idx, lse, dQ, dK, dV, stream=None
     return _call(
         "kmip_attn_bwd_deterministic", _ptr(dOut), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(lse), _ptr(dQ), _ptr(dK),
         _ptr(dV), _stream(stream), int(N), int(H), int(d), int(k), float(scale), int(dtype))
+
+
+def kmip_attn_gather(Q, K, V, idx, N, H, d, k, scale, out, lse, stream=None, dtype=None) -> int:
+    """Softmax and V gather over the given key sets (idx), scores recomputed."""
+    _check_cuda(Q, K, V, idx, out, lse)
+    if dtype is None:
+        dtype = dtype_code(Q.dtype)
+    return _call("kmip_attn_gather", _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), int(N), int(H),
+                 int(d), int(k), float(scale), _ptr(out), _ptr(lse), _stream(stream), int(dtype))
+
+
+def attn_gather(Q, K, V, idx, scale: float, stream=None):
+    """Returns (out, lse) of attention over the given sets idx [N, H, k]."""
+    N, H, d = Q.shape
+    out = torch.empty_like(Q)
+    lse = torch.empty((N, H), dtype=torch.float32, device=Q.device)
+    rc = kmip_attn_gather(Q, K, V, idx, N, H, d, idx.shape[-1], scale, out, lse, stream)
+    if rc:
+        raise KmipError(rc, "kmip_attn_gather")
+    return out, lse
 
 
 def kmip_get_status(stream=None) -> int:

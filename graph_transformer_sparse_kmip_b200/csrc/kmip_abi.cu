@@ -205,6 +205,26 @@ KMIP_EXPORT kmip_status_t kmip_attn_bwd_deterministic(const void* dOut, const vo
                        true);
 }
 
+KMIP_EXPORT kmip_status_t kmip_attn_gather(const void* Q, const void* K, const void* V,
+                                           const int32_t* idx, int64_t N, int H, int d, int k,
+                                           float scale, void* out, float* lse,
+                                           kmip_stream_t stream_, kmip_dtype_t dtype) {
+  kmip_status_t st = check_common(N, H, d, k, scale, dtype);
+  if (st != KMIP_OK) return st;
+  if (N == 0) return KMIP_OK;
+  if (!Q || !K || !V || !idx || !out || !lse) return KMIP_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
+    return KMIP_ERR_INVALID_ARG;
+  int* status = status_ptr();
+  if (!status) return KMIP_ERR_CUDA;
+  GatherArgs a{Q, K, V, idx, (int)N, H, d, k, scale, out, lse, status};
+  if (launch_gather(dtype, a, static_cast<cudaStream_t>(stream_)) != cudaSuccess) {
+    cudaGetLastError();
+    return KMIP_ERR_CUDA;
+  }
+  return KMIP_OK;
+}
+
 KMIP_EXPORT kmip_status_t kmip_get_status(kmip_stream_t stream_) {
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (cudaStreamSynchronize(stream) != cudaSuccess) {

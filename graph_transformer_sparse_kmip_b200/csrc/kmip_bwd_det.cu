@@ -203,6 +203,9 @@ gather_reduce_kernel(const T* __restrict__ Q, const T* __restrict__ dO,
       const uint32_t pos = p0 + rs;
       if (pos < hi) {
         const uint32_t e = vals[pos];
+#ifdef KMIP_DEBUG_BOUNDS
+        if ((int64_t)(e / (uint32_t)k) >= buckets) continue;  // not a (query, head) of [N, H]
+#endif
         const float2 c = coef[e];
         const int64_t row = (int64_t)(e / (uint32_t)k) * D;  // (query, head) row of [N, H, d]
         float q[VN], g[VN];

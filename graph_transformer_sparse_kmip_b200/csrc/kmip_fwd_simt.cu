@@ -131,6 +131,9 @@ fwd_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __res
       for (int t = 0; t < cnt; ++t) {
         const float p = expf(scale * ls[t * kThreads + x] - L);
         const int j = li[t * kThreads + x];
+#ifdef KMIP_DEBUG_BOUNDS
+        if (j < it.j0 || j >= it.j1) continue;  // cannot happen: keys come from [j0, j1)
+#endif
 #pragma unroll
         for (int c = 0; c < D; c += VN) {
           float f[VN];

@@ -654,20 +654,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         const uint32_t todo = __reduce_or_sync(0xffffffffu, mask);
         if (todo) {
-          if (!__any_sync(0xffffffffu, rn + __popc(mask) > NR)) {
-            // Every lane has room: predicated stores, no branch per group.
+          // Only the groups that some lane keeps issue their (predicated)
+          // stores: in the steady state a few of the eight.  The branch on
+          // a group's bit is warp-uniform and the loop is unrolled, so the
+          // scores stay statically indexed registers.
+          const bool room = !__any_sync(0xffffffffu, rn + __popc(mask) > NR);
 #pragma unroll
-            for (int g = 0; g < kBN / 16; ++g)
-              push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16, jt + g * 16);
-          } else {
-            // Some lane runs out of records within this tile: hand batches
-            // over between groups.
-#pragma unroll
-            for (int g = 0; g < kBN / 16; ++g) {
-              if (todo & (1u << g)) {  // warp-uniform
-                if (__any_sync(0xffffffffu, rn == NR)) hand_over(0);
-                push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16, jt + g * 16);
-              }
+          for (int g = 0; g < kBN / 16; ++g) {
+            if (todo & (1u << g)) {
+              const bool on = (mask >> g) & 1u;
+              // a lane whose buffer is full and keeps this group hands the
+              // batch over first (never when every lane had room)
+              if (!room && __any_sync(0xffffffffu, on && rn == NR)) hand_over(0);
+              push_if(on, v[g >> 1] + (g & 1) * 16, jt + g * 16);
             }
           }
           // Hand a batch over early once enough rows hold records and the
@@ -757,6 +756,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
           for (int u = 0; u < CW; ++u) o[u] = 0.f;
           for (int t = 0; t < cnt; ++t) {
+#ifdef KMIP_DEBUG_BOUNDS
+            if (Jf[t] < it.j0 || Jf[t] >= it.j1) {
+              record_status(p.status, KMIP_ERR_BAD_INDEX);
+              continue;
+            }
+#endif
             const float pw = expf(p.scale * Lf[t] - lse_v);
             const __nv_bfloat16* vr = p.V + (int64_t)Jf[t] * HD + h * D + c0;
 #pragma unroll

@@ -53,6 +53,18 @@ struct BwdArgs {
   DetBuffers det = {};  // keys != nullptr: write coefficients instead of scattering
 };
 
+struct GatherArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int32_t* idx;
+  int N, H, d, k;
+  float scale;
+  void* out;
+  float* lse;
+  int* status;
+};
+
 // Queries per work item of each forward kernel (the tensor-core forward
 // takes two 128-row Q tiles per item).
 constexpr int kSimtQueries = 128;
@@ -75,6 +87,9 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 bool fwd_tc_supported(int d, int k);
 
 cudaError_t launch_bwd(kmip_dtype_t dtype, const BwdArgs& a, cudaStream_t stream);
+
+// Softmax and V gather over given key sets (kmip_gather.cu).
+cudaError_t launch_gather(kmip_dtype_t dtype, const GatherArgs& a, cudaStream_t stream);
 
 // Deterministic backward: coefficients, a stable sort of the kept keys by
 // (key, head) and an in-order reduction per key (kmip_bwd_det.cu).  Takes

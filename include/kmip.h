@@ -157,6 +157,27 @@ kmip_status_t kmip_attn_fwd_diag(const void* Q, const void* K, const void* V,
                                  kmip_dtype_t dtype);
 
 /*
+ * Attention over given key sets: the softmax and V-gather stage of the
+ * forward on its own (k-Maximum Inner Product Attention for Graph
+ * Transformers ..., Abstract: once a query's k keys are chosen the layer is
+ * softmax attention over them).  For a caller that keeps a selection across
+ * calls, and the gather stage measured by itself.
+ *   Q, K, V        [N, H, d] of `dtype` (device).
+ *   idx            [N, H, k] int32 (device): the kept keys of each (query,
+ *                  head), -1 = padding (as kmip_attn_fwd writes it).  The
+ *                  scores of the kept keys are recomputed from Q and K.
+ *   out            [N, H, d] of `dtype` (device), overwritten.
+ *   lse            [N, H] fp32 (device), overwritten (-inf for a row whose
+ *                  entries are all -1).
+ * An idx entry outside [-1, N) records KMIP_ERR_BAD_INDEX on the device and
+ * is skipped.  Returns KMIP_OK, KMIP_ERR_INVALID_ARG, KMIP_ERR_UNSUPPORTED or
+ * KMIP_ERR_CUDA.
+ */
+kmip_status_t kmip_attn_gather(const void* Q, const void* K, const void* V, const int32_t* idx,
+                               int64_t N, int H, int d, int k, float scale, void* out,
+                               float* lse, kmip_stream_t stream, kmip_dtype_t dtype);
+
+/*
  * Backward pass.
  *   dOut           [N, H, d] of `dtype` (device): gradient of the loss w.r.t. out.
  *   Q, K, V        the forward's inputs; idx, lse the forward's outputs.
