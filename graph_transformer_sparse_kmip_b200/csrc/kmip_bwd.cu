@@ -13,9 +13,7 @@
 // 32 / (d / slice) kept rows at once with coalesced 16-byte loads.  Pass 1
 // recomputes s_j and dP_j for every kept key, pass 2 forms dS_j, accumulates
 // dQ in registers and scatters dK/dV rows with vector fp32 reductions
-// (red.global.add.v4.f32), one 16-byte reduction per lane per row.  The key
-// slices of the first passes stay in registers, so pass 2 reads no K row
-// again (up to 4 passes: k <= 32 at d = 32 bf16, k <= 64 at d = 16).
+// (red.global.add.v4.f32), one 16-byte reduction per lane per row.
 #include <math.h>
 
 #include "kmip_internal.h"
@@ -25,14 +23,13 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kKmax = 64;
-constexpr int kCache = 4;  // passes whose K slices stay in registers between the two passes
 
 // DET: instead of scattering into dK/dV, write for every kept key its
 // coefficients (p_j, scale dS_j), its (key, head) bucket as a sort key and
 // its position in idx as the sort value, and count the bucket's entries;
 // the deterministic reduction (kmip_bwd_det.cu) sums them per key.
 template <typename T, int D, bool DET>
-__global__ void __launch_bounds__(kWarps * 32, 4)
+__global__ void __launch_bounds__(kWarps * 32)
 bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restrict__ K,
            const T* __restrict__ V, const int32_t* __restrict__ idx,
            const float* __restrict__ lse, float* __restrict__ dQ, float* __restrict__ dK,
@@ -55,17 +52,15 @@ bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restric
   for (int64_t pr = (int64_t)blockIdx.x * kWarps + warp; pr < pairs;
        pr += (int64_t)gridDim.x * kWarps) {
     const int64_t base = pr * D;  // row (i, h) of [N, H, d]
-    const int64_t hoff = base % HD;
     float q[VN], go[VN];
     VT::load(Q + base + cs, q);
     VT::load(dO + base + cs, go);
     const float L = lse[pr];
     const int32_t* ir = idx + pr * k;
 
-    // Pass 1: p_j and dP_j of every kept key.  The K slices of the first
-    // kCache passes stay in registers for pass 2.
+    // Pass 1: p_j and dP_j of every kept key.
     float Dsum = 0.f;
-    auto pass1 = [&](int ps, typename VT::Raw& kraw) -> int {
+    for (int ps = 0; ps < npass; ++ps) {
       const int t = ps * RPP + rs;
       int j = t < k ? ir[t] : -1;
       if (j >= N || j < -1) {
@@ -75,9 +70,8 @@ bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restric
       float s = 0.f, dp = 0.f;
       if (j >= 0) {
         float kv[VN], vv[VN];
-        kraw = VT::load_raw(K + (int64_t)j * HD + hoff + cs);
-        VT::load(V + (int64_t)j * HD + hoff + cs, vv);
-        VT::unpack(kraw, kv);
+        VT::load(K + (int64_t)j * HD + (base % HD) + cs, kv);
+        VT::load(V + (int64_t)j * HD + (base % HD) + cs, vv);
 #pragma unroll
         for (int u = 0; u < VN; ++u) {
           s = fmaf(q[u], kv[u], s);
@@ -102,18 +96,6 @@ bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restric
         }
       }
       Dsum = fmaf(p, dp, Dsum);  // identical in the LPR lanes of a row
-      return j;
-    };
-    typename VT::Raw kc[kCache];
-    int jc[kCache];
-#pragma unroll
-    for (int ps = 0; ps < kCache; ++ps) {
-      jc[ps] = -1;
-      if (ps < npass) jc[ps] = pass1(ps, kc[ps]);
-    }
-    for (int ps = kCache; ps < npass; ++ps) {
-      typename VT::Raw kraw;
-      pass1(ps, kraw);
     }
 #pragma unroll
     for (int o = LPR; o < 32; o <<= 1) Dsum += __shfl_xor_sync(0xffffffffu, Dsum, o);
@@ -123,33 +105,29 @@ bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restric
     float dq[VN];
 #pragma unroll
     for (int u = 0; u < VN; ++u) dq[u] = 0.f;
-    auto pass2 = [&](int t, int j, const typename VT::Raw& kraw) {
-      float kv[VN];
-      VT::unpack(kraw, kv);
-      const float p = sp[warp][t];
-      const float ds = p * (sdp[warp][t] - Dsum);
-      const int64_t kb = (int64_t)j * HD + hoff + cs;
-#pragma unroll
-      for (int u = 0; u < VN; ++u) dq[u] = fmaf(ds, kv[u], dq[u]);
-      const float a = scale * ds;
-      if constexpr (DET) {
-        if ((lane % LPR) == 0) det.coef[pr * k + t] = make_float2(p, a);
-      } else {
-#pragma unroll
-        for (int u = 0; u < VN; u += 4) {
-          red_add_v4(dK + kb + u, a * q[u], a * q[u + 1], a * q[u + 2], a * q[u + 3]);
-          red_add_v4(dV + kb + u, p * go[u], p * go[u + 1], p * go[u + 2], p * go[u + 3]);
-        }
-      }
-    };
-#pragma unroll
-    for (int ps = 0; ps < kCache; ++ps)
-      if (ps < npass && jc[ps] >= 0) pass2(ps * RPP + rs, jc[ps], kc[ps]);
-    for (int ps = kCache; ps < npass; ++ps) {
+    for (int ps = 0; ps < npass; ++ps) {
       const int t = ps * RPP + rs;
       int j = t < k ? ir[t] : -1;
       if (j >= N || j < -1) j = -1;
-      if (j >= 0) pass2(t, j, VT::load_raw(K + (int64_t)j * HD + hoff + cs));
+      if (j >= 0) {
+        const float p = sp[warp][t];
+        const float ds = p * (sdp[warp][t] - Dsum);
+        const int64_t kb = (int64_t)j * HD + (base % HD) + cs;
+        float kv[VN];
+        VT::load(K + kb, kv);
+#pragma unroll
+        for (int u = 0; u < VN; ++u) dq[u] = fmaf(ds, kv[u], dq[u]);
+        const float a = scale * ds;
+        if constexpr (DET) {
+          if ((lane % LPR) == 0) det.coef[pr * k + t] = make_float2(p, a);
+        } else {
+#pragma unroll
+          for (int u = 0; u < VN; u += 4) {
+            red_add_v4(dK + kb + u, a * q[u], a * q[u + 1], a * q[u + 2], a * q[u + 3]);
+            red_add_v4(dV + kb + u, p * go[u], p * go[u + 1], p * go[u + 2], p * go[u + 3]);
+          }
+        }
+      }
     }
 #pragma unroll
     for (int o = LPR; o < 32; o <<= 1) {

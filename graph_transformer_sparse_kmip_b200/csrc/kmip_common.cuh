@@ -31,20 +31,14 @@ struct Vec;  // 16-byte vector of T, widened to fp32
 template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int N = 8;
-  using Raw = uint4;  // the 16 bytes as loaded (8 packed bf16)
-  __device__ __forceinline__ static Raw load_raw(const __nv_bfloat16* p) {
-    return __ldg(reinterpret_cast<const uint4*>(p));
-  }
-  __device__ __forceinline__ static void unpack(const Raw& u, float* f) {
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* f) {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       f[2 * t] = __uint_as_float(w[t] << 16);
       f[2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
     }
-  }
-  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* f) {
-    unpack(load_raw(p), f);
   }
   __device__ __forceinline__ static void store(__nv_bfloat16* p, const float* f) {
     uint32_t w[4];
@@ -60,15 +54,9 @@ struct Vec<__nv_bfloat16> {
 template <>
 struct Vec<float> {
   static constexpr int N = 4;
-  using Raw = float4;
-  __device__ __forceinline__ static Raw load_raw(const float* p) {
-    return __ldg(reinterpret_cast<const float4*>(p));
-  }
-  __device__ __forceinline__ static void unpack(const Raw& u, float* f) {
-    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
-  }
   __device__ __forceinline__ static void load(const float* p, float* f) {
-    unpack(load_raw(p), f);
+    float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
   }
   __device__ __forceinline__ static void store(float* p, const float* f) {
     *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);

@@ -33,14 +33,14 @@
 //   warps 12..19  inserters, one per filter warp and one thread per row: they
 //                 take the handed-over buffers in order, insert every
 //                 recorded score that beats the row's threshold into the
-//                 row's sorted top-k list (a branch-free compare-exchange
-//                 chain over a list held in registers for k <= 16; binary
-//                 search and shift in shared memory for larger k; lists of
-//                 16, 32, 48 or 64 slots), publish the new threshold, which
-//                 the filter reads every tile, and after an item's last
-//                 batch compute the softmax over the kept scores, lse, and the
-//                 weighted sum of the kept V rows (16-byte loads) while the
-//                 filters already work on the next item.
+//                 row's top-k (k <= 16: a sorted list held in registers for
+//                 the whole item, candidates moving up from the last slot;
+//                 larger k: a heap in shared memory with the worst entry at
+//                 the root; 16, 32, 48 or 64 slots), publish the new
+//                 threshold, which the filter reads every tile, and after an
+//                 item's last batch compute the softmax over the kept scores,
+//                 lse, and the weighted sum of the kept V rows (16-byte loads)
+//                 while the filters already work on the next item.
 // The warpgroups rebalance their registers at the start (setmaxnreg): the
 // producer/MMA warpgroup and the inserters give some up, and the filters,
 // which hold a tile's scores, take them (32 / 160 / 64 per thread: the split
@@ -174,8 +174,10 @@ __device__ __forceinline__ float max16(const float* x) {
 
 // A row's top-k list is its line of shared memory: scores ls[..] and keys
 // li[..].  For KCAP == kRegK it is a sorted list of kRegK slots, larger score
-// first: the first kRegK - k slots hold +inf sentinels and the k real entries
-// follow, so the k-th best is always the last slot.  For larger KCAP the k
+// first, kept in the insert thread's registers during an item and written
+// here for the softmax and gather: the first kRegK - k slots hold +inf
+// sentinels and the k real entries follow, so the k-th best is always the
+// last slot.  For larger KCAP the k
 // entries form a binary heap with the worst entry at the root (slot 0):
 // entry a is worse than entry b when a's score is smaller, or equal with a
 // larger key; the root's score is the row's threshold.  Unused entries hold
@@ -287,27 +289,19 @@ __device__ __forceinline__ bool next_candidate(uint64_t& m, const float* rs, con
   return false;
 }
 
-// Insertion for k <= kRegK: the list is held in registers and every lane
-// takes one candidate per round.  A candidate beats the last slot (the k-th
-// best), so it replaces it and then moves up while it is strictly larger
-// than the entry before it; the rounds stop moving as soon as no lane's
-// candidate moves, which in the steady state (candidates just above the
-// threshold) is after a step or two.  Records are visited in key order, so
-// an equal score stays behind the entries already listed.  Returns the new
-// threshold.
+// Insertion for k <= kRegK: the insert warp keeps the row's list in
+// registers for the whole item and takes one candidate per lane per round.
+// A candidate beats the last slot (the k-th best), so it replaces it and
+// then moves up while it is strictly larger than the entry before it; a
+// round stops as soon as no lane's candidate moves, which in the steady
+// state (candidates just above the threshold) is after a step or two.
+// Records are visited in key order, so an equal score stays behind the
+// entries already listed.  Returns the new threshold.
 template <int NREC>
-__device__ __forceinline__ float insert_regs(float* ls, int* li, const float* rs, const int* rj,
-                                             int rn, float thr) {
+__device__ __forceinline__ float insert_in_regs(float (&L)[kRegK], int (&J)[kRegK], const float* rs,
+                                                const int* rj, int rn, float thr) {
   uint64_t m = record_bits<NREC>(rs, rn, thr);
-  if (!__any_sync(0xffffffffu, m != 0)) return thr;
-  float L[kRegK];
-  int J[kRegK];
-#pragma unroll
-  for (int t = 0; t < kRegK; ++t) {
-    L[t] = ls[t];
-    J[t] = li[t];
-  }
-  while (true) {
+  while (__any_sync(0xffffffffu, m != 0)) {
     float s = -INFINITY;
     int j = -1;
     const bool have = next_candidate(m, rs, rj, thr, s, j);
@@ -329,12 +323,6 @@ __device__ __forceinline__ float insert_regs(float* ls, int* li, const float* rs
     }
     thr = L[kRegK - 1];
   }
-#pragma unroll
-  for (int t = 0; t < kRegK; ++t) {
-    ls[t] = L[t];
-    li[t] = J[t];
-  }
-  __syncwarp();
   return thr;
 }
 
@@ -658,15 +646,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           // stores: in the steady state a few of the eight.  The branch on
           // a group's bit is warp-uniform and the loop is unrolled, so the
           // scores stay statically indexed registers.
-          const bool room = !__any_sync(0xffffffffu, rn + __popc(mask) > NR);
+          if (!__any_sync(0xffffffffu, rn + __popc(mask) > NR)) {
 #pragma unroll
-          for (int g = 0; g < kBN / 16; ++g) {
-            if (todo & (1u << g)) {
-              const bool on = (mask >> g) & 1u;
-              // a lane whose buffer is full and keeps this group hands the
-              // batch over first (never when every lane had room)
-              if (!room && __any_sync(0xffffffffu, on && rn == NR)) hand_over(0);
-              push_if(on, v[g >> 1] + (g & 1) * 16, jt + g * 16);
+            for (int g = 0; g < kBN / 16; ++g)
+              if (todo & (1u << g)) push_if((mask >> g) & 1u, v[g >> 1] + (g & 1) * 16, jt + g * 16);
+          } else {
+            // some lane runs out of records within this tile: hand batches
+            // over between groups
+#pragma unroll
+            for (int g = 0; g < kBN / 16; ++g) {
+              if (todo & (1u << g)) {
+                const bool on = (mask >> g) & 1u;
+                if (__any_sync(0xffffffffu, on && rn == NR)) hand_over(0);
+                push_if(on, v[g >> 1] + (g & 1) * 16, jt + g * 16);
+              }
             }
           }
           // Hand a batch over early once enough rows hold records and the
@@ -706,7 +699,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const WorkItem it = p.items[w % count];
       const bool tile_on = mt == 0 || (it.q1 - it.q0) > kBM;
       const int i = it.q0 + mt * kBM + row;
-      list_reset<KCAP>(L, J, p.k);
+      float RL[kRegK];
+      int RJ[kRegK];
+      if constexpr (KCAP == kRegK) {
+#pragma unroll
+        for (int t = 0; t < kRegK; ++t) {
+          RL[t] = t < kRegK - p.k ? INFINITY : -INFINITY;
+          RJ[t] = -1;
+        }
+      } else {
+        list_reset<KCAP>(L, J, p.k);
+      }
       float thr = -INFINITY;
       ++item_no;
       for (;;) {
@@ -720,8 +723,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int flags = bflag[cb * kFilterWarps + f];
         const float* rs = rec_s + (cb * kRows + et) * RS;
         const int* rj = rec_j + cb * NR * kRows + et;
-        if (KCAP == kRegK)
-          thr = insert_regs<NR>(L, J, rs, rj, rn, thr);
+        if constexpr (KCAP == kRegK)
+          thr = insert_in_regs<NR>(RL, RJ, rs, rj, rn, thr);
         else
           thr = insert_heap<NR>(L, J, rs, rj, rn, thr, p.k);
         {
@@ -737,6 +740,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (flags & 1) break;
       }
       if (!ok) break;
+      if constexpr (KCAP == kRegK) {
+#pragma unroll
+        for (int t = 0; t < kRegK; ++t) {
+          L[t] = RL[t];
+          J[t] = RJ[t];
+        }
+      }
       if (tile_on && i < it.q1) {
         if (KCAP != kRegK) heap_to_sorted(L, J, p.k);
         const float* Lf = L + first_slot<KCAP>(p.k);

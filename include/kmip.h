@@ -201,7 +201,9 @@ kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K, cons
  * positions in idx, so repeated calls on the same inputs return identical
  * bits.  Takes O(N H k) scratch (about 28 bytes per kept key plus 4 per
  * (node, head)) from the stream-ordered allocator of the current device and
- * releases it on the same stream.  Returns KMIP_ERR_UNSUPPORTED when
+ * releases it on the same stream; it raises the release threshold of the
+ * device's default memory pool to that size (never lowers it), so repeated
+ * calls reuse the memory instead of mapping it anew each time.  Returns KMIP_ERR_UNSUPPORTED when
  * N H k >= 2^32 - 1 or the sort's scans would exceed 2^24 entries
  * (N H k > about 2.7e8); otherwise as kmip_attn_bwd.
  */
