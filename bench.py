@@ -1,7 +1,8 @@
 """Benchmark: k-MIP attention query-heads/s, forward and forward+backward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gmm_n100000] [--k 15]
+                    [--workload gmm_n100000] [--k 15] [--no-configs] [--no-baselines]
+                    [--no-k-sweep] [--no-e2e] [--no-cpu-baseline]
 
 One step is the whole hot path over one batch: the forward (work list,
 fused score + top-k + softmax + V gather) and the backward (recompute,
@@ -11,10 +12,16 @@ summed over ranks.  With N > 1 GPUs (torchrun) every rank runs its own
 independent batch (a different seed) -- there is no data-path collective;
 the only collectives are the barriers and the max-over-ranks of the time.
 
-Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
-on the launching stream; between steps a 256 MiB buffer is written to flush
-the L2 (126 MB), outside the events.  A barrier and a device synchronise
-bracket the whole timed loop.  One JSON line is printed by rank 0.
+Timing: W untimed warm-up steps, then K steps, each phase bracketed by CUDA
+events on the launching stream; between steps a 256 MiB buffer is written to
+flush the L2 (126 MB), outside the events.  A barrier and a device
+synchronise bracket the whole timed loop.  Besides the headline step the line
+carries: per-step times and SM clocks, the backward's and the gather stage's
+GB/s, the deterministic backward, the k sweep, the other four workloads
+(`configs`), torch's full attention and dense top-k on the same inputs with
+the Figure 8 diagnostics (`baselines`), the end-to-end run from pinned host
+buffers (`e2e`) and the fp64 oracle on the host cores (`cpu_baseline`).
+One JSON line is printed by rank 0.
 """
 from __future__ import annotations
 
