@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTE
                 6: "KMIP_ERR_BAD_INDEX", 7: "KMIP_ERR_SCRATCH_LIMIT"}
 EXPORTED = ("kmip_attn_fwd", "kmip_attn_fwd_noalloc", "kmip_attn_fwd_diag", "kmip_attn_bwd",
             "kmip_attn_bwd_deterministic", "kmip_attn_gather", "kmip_get_status",
-            "kmip_error_string",
+            "kmip_scratch_usage", "kmip_error_string",
             "kmip_fwd_path", "kmip_version")
 
 _lib = None
@@ -63,6 +63,8 @@ def load() -> ctypes.CDLL:
     lib.kmip_attn_gather.restype = I32
     lib.kmip_get_status.argtypes = [P]
     lib.kmip_get_status.restype = I32
+    lib.kmip_scratch_usage.argtypes = [P, P, I32]
+    lib.kmip_scratch_usage.restype = I32
     lib.kmip_error_string.argtypes = [I32]
     lib.kmip_error_string.restype = ctypes.c_char_p
     lib.kmip_test_wait_timeout.argtypes = [P, I32]
@@ -218,6 +220,16 @@ def kmip_get_status(stream=None) -> int:
 
 def kmip_error_string(code: int) -> str:
     return load().kmip_error_string(int(code)).decode()
+
+
+def kmip_scratch_usage(reset_high: bool = False):
+    """(reserved, used_high) bytes of the library's scratch pool on the
+    current device."""
+    r, h = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    rc = load().kmip_scratch_usage(ctypes.byref(r), ctypes.byref(h), int(bool(reset_high)))
+    if rc:
+        raise KmipError(rc, "kmip_scratch_usage")
+    return int(r.value), int(h.value)
 
 
 def kmip_version() -> int:

@@ -1,5 +1,6 @@
 // kmip_abi.cu -- the C ABI of libkmip (declared in include/kmip.h): argument
-// checks, the per-device status word, work-list scratch and kernel dispatch.
+// checks, the per-device status word, the library's scratch pool and kernel
+// dispatch.
 #include <math.h>
 
 #include <mutex>
@@ -24,6 +25,8 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int* g_status_ptr[kMaxDevices] = {};
 int g_sm_count[kMaxDevices] = {};
+cudaMemPool_t g_pool[kMaxDevices] = {};
+uint64_t g_pool_keep[kMaxDevices] = {};
 
 }  // namespace
 
@@ -57,6 +60,72 @@ kmip_status_t check_common(int64_t N, int H, int d, int k, float scale, kmip_dty
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The library's own stream-ordered memory pool on the current device.  It
+// keeps, between calls, the most memory it has held (its release threshold
+// follows its largest reservation), so a loop of calls maps device memory
+// once instead of on every call, and it leaves the device's default pool,
+// which other code in the process may use, alone.
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_pool[dev]) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.handleTypes = cudaMemHandleTypeNone;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      const cudaError_t e = cudaMemPoolCreate(&g_pool[dev], &props);
+      if (e != cudaSuccess) {
+        g_pool[dev] = nullptr;
+        cudaGetLastError();
+        return e;
+      }
+    }
+    pool = g_pool[dev];
+  }
+  const cudaError_t e = cudaMallocFromPoolAsync(p, bytes, pool, stream);
+  if (e == cudaSuccess) {
+    // keep all that the pool holds now: trimming to the request alone would
+    // still return the last, partly used block of the pool's reservation
+    std::lock_guard<std::mutex> lock(g_mu);
+    uint64_t r = 0;
+    if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent, &r) == cudaSuccess &&
+        r > g_pool_keep[dev] &&
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &r) == cudaSuccess)
+      g_pool_keep[dev] = r;
+    cudaGetLastError();
+  }
+  return e;
+}
+
+// Reserved and high-water bytes of the library's pool on the current device
+// (zeros before its first allocation).
+cudaError_t scratch_usage(uint64_t* reserved, uint64_t* used_high, bool reset_high) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  uint64_t r = 0, h = 0;
+  cudaMemPool_t pool = g_pool[dev];
+  if (pool) {
+    if (reset_high) {
+      uint64_t zero = 0;
+      if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &zero) != cudaSuccess)
+        return cudaGetLastError();
+    }
+    if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent, &r) != cudaSuccess ||
+        cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &h) != cudaSuccess)
+      return cudaGetLastError();
+  }
+  if (reserved) *reserved = r;
+  if (used_high) *used_high = h;
+  return cudaSuccess;
+}
 
 int device_sm_count() {
   int dev = 0;
@@ -103,7 +172,7 @@ kmip_status_t attn_fwd_impl(const void* Q, const void* K, const void* V,
   // Work-list scratch: [count (16 B)] [items], stream-ordered.
   void* scratch = nullptr;
   const size_t bytes = 16 + sizeof(WorkItem) * (size_t)max_items;
-  if (cudaMallocAsync(&scratch, bytes, stream) != cudaSuccess) {
+  if (scratch_alloc(&scratch, bytes, stream) != cudaSuccess) {
     cudaGetLastError();
     return KMIP_ERR_CUDA;
   }
@@ -243,6 +312,12 @@ KMIP_EXPORT kmip_status_t kmip_get_status(kmip_stream_t stream_) {
   return static_cast<kmip_status_t>(h);
 }
 
+KMIP_EXPORT kmip_status_t kmip_scratch_usage(uint64_t* reserved, uint64_t* used_high,
+                                             int reset_high) {
+  return kmip::scratch_usage(reserved, used_high, reset_high != 0) == cudaSuccess ? KMIP_OK
+                                                                                  : KMIP_ERR_CUDA;
+}
+
 KMIP_EXPORT const char* kmip_error_string(kmip_status_t s) {
   switch (s) {
     case KMIP_OK: return "KMIP_OK: success";
@@ -263,4 +338,4 @@ KMIP_EXPORT int kmip_fwd_path(int d, int k, kmip_dtype_t dtype) {
   return dtype == KMIP_BF16 && fwd_tc_supported(d, k) ? 1 : 0;
 }
 
-KMIP_EXPORT int kmip_version(void) { return 100; }
+KMIP_EXPORT int kmip_version(void) { return 200; }

@@ -286,21 +286,8 @@ cudaError_t launch_bwd_deterministic(kmip_dtype_t dtype, const BwdArgs& a_in, cu
   const size_t o_coef = take(sizeof(float2) * E), o_k0 = take(4 * E), o_v0 = take(4 * E),
                o_k1 = take(4 * E), o_v1 = take(4 * E), o_cnt = take(4 * (NB + 1)),
                o_hist = take(4 * hist_n), o_sums = take(4 * sums_n);
-  // Keep at least this much in the device's default pool between calls, so
-  // that a training loop does not map fresh memory on every backward.
-  int dev = 0;
-  cudaMemPool_t pool;
-  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
-    uint64_t keep = 0;
-    if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) == cudaSuccess &&
-        keep < bytes) {
-      keep = bytes;
-      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-    }
-  }
-  cudaGetLastError();
   char* scratch = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), bytes, stream) != cudaSuccess)
+  if (scratch_alloc(reinterpret_cast<void**>(&scratch), bytes, stream) != cudaSuccess)
     return cudaErrorMemoryAllocation;
   float2* coef = reinterpret_cast<float2*>(scratch + o_coef);
   uint32_t* keys[2] = {reinterpret_cast<uint32_t*>(scratch + o_k0),

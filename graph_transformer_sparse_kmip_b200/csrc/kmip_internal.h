@@ -93,10 +93,15 @@ cudaError_t launch_gather(kmip_dtype_t dtype, const GatherArgs& a, cudaStream_t 
 
 // Deterministic backward: coefficients, a stable sort of the kept keys by
 // (key, head) and an in-order reduction per key (kmip_bwd_det.cu).  Takes
-// its scratch from the stream-ordered allocator.
+// its scratch from the library's pool (scratch_alloc).
 cudaError_t launch_bwd_deterministic(kmip_dtype_t dtype, const BwdArgs& a, cudaStream_t stream);
 
 int device_sm_count();
+
+// Stream-ordered allocation from the library's own memory pool on the
+// current device (kmip_abi.cu); free with cudaFreeAsync on the same stream.
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream);
+cudaError_t scratch_usage(uint64_t* reserved, uint64_t* used_high, bool reset_high);
 
 // Per-device status word address (nullptr if it cannot be resolved).
 int* status_ptr();

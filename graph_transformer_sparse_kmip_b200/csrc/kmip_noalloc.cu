@@ -1,7 +1,7 @@
 // kmip_noalloc.cu -- a forward entry point that allocates no device memory.
 //
-// kmip_attn_fwd takes its work list from the stream-ordered allocator on
-// every call.  Some callers cannot allow that: a framework whose own pool
+// kmip_attn_fwd takes its work list from the library's stream-ordered memory
+// pool on every call.  Some callers cannot allow that: a framework whose own pool
 // has reserved the GPU's memory up front, a process on a driver or
 // virtualised device without stream-ordered memory pools, or a latency-
 // critical loop that must not enter the allocator after start-up.

@@ -31,8 +31,12 @@
  * tensor memory / registers only.  The library's own device memory is a
  * work list of O(N / q + G) 16-byte items per forward call (q = 256 queries
  * per item on the tensor-core path, 128 otherwise; the same items serve
- * every head), taken from the stream-ordered allocator of the current
- * device and released on the same stream.
+ * every head), and the deterministic backward's sort scratch.  Both are
+ * stream-ordered allocations from a memory pool the library creates on each
+ * device it is called on (cudaMemPoolCreate; the device's default pool is
+ * not touched), released on the same stream.  The pool keeps, between
+ * calls, the most memory it has reserved so far (about the largest scratch
+ * taken from it), so a loop of calls maps device memory only once.
  *
  * Conventions common to every call:
  *   - All tensor pointers are DEVICE pointers on the current CUDA device
@@ -109,7 +113,7 @@ kmip_status_t kmip_attn_fwd(const void* Q, const void* K, const void* V,
  * pages: this is an interface variant for callers, not part of the method.)
  *
  * Same arguments, outputs and results as kmip_attn_fwd.  kmip_attn_fwd
- * takes its work list from the stream-ordered allocator on each call; this
+ * takes its work list from the library's memory pool on each call; this
  * variant is for callers that cannot let a library allocate: a framework
  * whose own memory pool already holds the GPU's memory, a driver or
  * virtualised device without stream-ordered memory pools, or a loop that
@@ -200,10 +204,8 @@ kmip_status_t kmip_attn_bwd(const void* dOut, const void* Q, const void* K, cons
  * dV rows are summed by one warp over its queries in the order of their
  * positions in idx, so repeated calls on the same inputs return identical
  * bits.  Takes O(N H k) scratch (about 28 bytes per kept key plus 4 per
- * (node, head)) from the stream-ordered allocator of the current device and
- * releases it on the same stream; it raises the release threshold of the
- * device's default memory pool to that size (never lowers it), so repeated
- * calls reuse the memory instead of mapping it anew each time.  Returns KMIP_ERR_UNSUPPORTED when
+ * (node, head)) from the library's memory pool (see Memory above) and
+ * releases it on the same stream.  Returns KMIP_ERR_UNSUPPORTED when
  * N H k >= 2^32 - 1 or the sort's scans would exceed 2^24 entries
  * (N H k > about 2.7e8); otherwise as kmip_attn_bwd.
  */
@@ -229,6 +231,17 @@ kmip_status_t kmip_get_status(kmip_stream_t stream);
  * logic; touches no device.
  */
 int kmip_fwd_path(int d, int k, kmip_dtype_t dtype);
+
+/*
+ * The library's scratch memory on the current device (see Memory above):
+ * *reserved = device memory the library's pool holds now (in use or kept
+ * for the next call), *used_high = the most it had in use at once since the
+ * pool was created or since the last call with reset_high != 0 (which
+ * restarts that count from what is in use now).  Both are 0 before the
+ * first allocating call on the device.  Either pointer may be NULL.
+ * Returns KMIP_OK, or KMIP_ERR_CUDA if the pool could not be queried.
+ */
+kmip_status_t kmip_scratch_usage(uint64_t* reserved, uint64_t* used_high, int reset_high);
 
 /* Static, human-readable name of a status code (never NULL). */
 const char* kmip_error_string(kmip_status_t status);
