@@ -13,9 +13,11 @@ independent batch (a different seed) -- there is no data-path collective;
 the only collectives are the barriers and the max-over-ranks of the time.
 
 Timing: W untimed warm-up steps, then K steps, each phase bracketed by CUDA
-events on the launching stream; between steps a 256 MiB buffer is written to
-flush the L2 (126 MB), outside the events.  A barrier and a device
-synchronise bracket the whole timed loop.  Besides the headline step the line
+events on the launching stream; between steps, outside the events, a 256 MiB
+buffer is written to flush the L2 (126 MB) and a ~5 ms device-side spin holds
+the stream until the step's launches are queued (a host stall then delays
+the spin, not the timed kernels).  A barrier and a device synchronise
+bracket the whole timed loop.  Besides the headline step the line
 carries: per-step times and SM clocks, the backward's and the gather stage's
 GB/s, the deterministic backward, the k sweep, the other four workloads
 (`configs`), torch's full attention and dense top-k on the same inputs with
@@ -26,6 +28,7 @@ One JSON line is printed by rank 0.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -115,9 +118,12 @@ def _traffic(kernel_key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling.  The sampler starts before the
+    warm-up (its start-up costs host time and driver calls) and the summary
+    keeps the samples whose timestamps fall inside the timed window
+    (mark_start / mark_end)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -130,6 +136,15 @@ class ClockSampler:
         except Exception:
             pass
         self.proc = None
+        self.window = None
+        self.lines = []
+
+    def mark_start(self):
+        self.window = [datetime.datetime.now(), None]
+
+    def mark_end(self):
+        if self.window:
+            self.window[1] = datetime.datetime.now()
 
     def __enter__(self):
         try:
@@ -152,29 +167,61 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    def _rows(self):
+        rows = []
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(f[2]), float(f[3]), f[6:10]))
             except ValueError:
                 continue
-            for nm, v in zip(names, f[5:9]):
+        return rows
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = self._rows()
+        window = "timed region"
+        if self.window and self.window[1]:
+            # a sample describes the 100 ms before it: keep those that end
+            # inside the window, and the first one after it
+            a, b = self.window
+            inside = [r for r in rows if a <= r[0] <= b]
+            after = [r for r in rows if r[0] > b][:1]
+            sel = inside + after
+            if not sel:
+                sel, window = rows, "whole run (no sample in the timed region)"
+        else:
+            sel, window = rows, "whole run"
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        reasons = set()
+        for r in sel:
+            for nm, v in zip(names, r[3]):
                 if v.lower() == "active":
                     reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(r[1] for r in sel), "sm_max_mhz": sel[-1][2],
+                "reasons": sorted(reasons), "samples": len(sel), "window": window}
 
 
 def _flush(buf):
     buf.add_(1)  # read + write 256 MiB: evicts the 126 MB L2
+
+
+GATE_CYCLES = 10_000_000  # about 5 ms at 1.97 GHz
+
+
+def _flush_and_gate(buf):
+    """Between timed steps, outside the events: flush the L2, then hold the
+    stream in a short device-side spin, so that the step's start event and
+    launches are all queued before the device reaches them.  A host stall
+    (another process on the host's cores, the sampler's start-up) then
+    delays the spin, not the timed kernels: the events measure device work
+    alone."""
+    _flush(buf)
+    torch.cuda._sleep(GATE_CYCLES)
 
 
 class SmClock:
@@ -258,18 +305,19 @@ class Case:
 
 def time_case(case, stream, steps, warmup, flush, clock=None, k=None, idx=None):
     """Per-step device times (ms) of the forward and the backward, each
-    bracketed by CUDA events on the launching stream, the L2 flushed
-    between steps outside the events; the SM clock read after every step."""
+    bracketed by CUDA events on the launching stream (torch's current
+    stream), the L2 flushed and the stream gated between steps outside the
+    events; the SM clock read after every step."""
     fwd_ms, bwd_ms, mhz = [], [], []
     for it in range(warmup + steps):
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        _flush_and_gate(flush)
         e0.record(stream)
         case.fwd(stream, k, idx)
         e1.record(stream)
         if case.bwd:
             case.bwd_call(stream, k, idx)
         e2.record(stream)
-        _flush(flush)
         torch.cuda.synchronize()
         if it >= warmup:
             fwd_ms.append(e0.elapsed_time(e1))
@@ -323,6 +371,7 @@ def run_ours(args, ws, rank, local):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     clock = SmClock(dev)
 
+    clk = ClockSampler(dev).__enter__()
     for _ in range(args.warmup):
         case.fwd(stream)
         case.bwd_call(stream)
@@ -333,11 +382,14 @@ def run_ours(args, ws, rank, local):
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(dev) as clk:
-        fwd_ms, bwd_ms, mhz = time_case(case, stream, args.steps, 0, flush, clock)
-        torch.cuda.synchronize()
-        if ws > 1:
-            torch.distributed.barrier()
+    clk.mark_start()
+    fwd_ms, bwd_ms, mhz = time_case(case, stream, args.steps, 0, flush, clock)
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    clk.mark_end()
+    time.sleep(0.15)  # one more sample after the window
+    clk.__exit__(None, None, None)
     binding.check_status()
     tot_ms = [a + b for a, b in zip(fwd_ms, bwd_ms)]
     t_fwd, t_bwd, t_tot = max_over_ranks([sum(fwd_ms), sum(bwd_ms), sum(tot_ms)], ws, dev)
@@ -361,7 +413,7 @@ def run_ours(args, ws, rank, local):
     gat_ms = []
     o_g, l_g = torch.empty_like(case.out), torch.empty_like(case.lse)
     for it in range(3 + max(3, args.steps // 2)):
-        _flush(flush)
+        _flush_and_gate(flush)
         a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a_.record(stream)
         rc = binding.kmip_attn_gather(g["Q"], g["K"], g["V"], case.idx, N, H, d, k, scale, o_g,
@@ -376,7 +428,7 @@ def run_ours(args, ws, rank, local):
     # the deterministic backward (sorted gather, no atomics) on the same step
     det_ms = []
     for it in range(3 + max(3, args.steps // 2)):
-        _flush(flush)
+        _flush_and_gate(flush)
         a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a_.record(stream)
         rc = binding.kmip_attn_bwd_deterministic(g["dO"], g["Q"], g["K"], g["V"], case.idx,
@@ -510,7 +562,7 @@ def run_ours(args, ws, rank, local):
         "config": {"workload": w.name, "N": N, "H": H, "d": d, "k": k,
                    "graphs": int(inp["offsets"].numel() - 1), "keys": w.values,
                    "step": "fwd+bwd", "parallelism": f"independent batch per GPU x{ws}",
-                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+                   "l2": "flushed between steps (256 MiB write, then a 5 ms device-side gate; both outside the timed events)"},
         "fwd": {"value": fwd_value, "unit": UNIT, "ms_per_step": ms_fwd},
         "roofline": {"bound": "tensor", "kernel": "forward (score + top-k + softmax + gather)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -578,7 +630,7 @@ def comparison_baselines(case, stream, flush, reps=3):
     def timed(fn):
         ts = []
         for it in range(reps + 1):
-            _flush(flush)
+            _flush_and_gate(flush)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             fn()
