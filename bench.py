@@ -773,7 +773,10 @@ def run_reference(args, ws, rank):
         "sample_pairs_per_step": statistics.mean(pairs),
         "full_step_ms_extrapolated": N * H / value * 1e3,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[-1]["cores"],
-                         "kind": "oracle", "sample": samples[-1]["sample"] + " per step"},
+                         "kind": "oracle",
+                         "sample": f"{statistics.mean(pairs):.0f} (query, head) pairs per step on "
+                                   f"average over {len(pairs)} steps (last step: "
+                                   + samples[-1]["sample"] + ")"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
