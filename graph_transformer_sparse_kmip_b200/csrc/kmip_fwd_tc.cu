@@ -36,8 +36,8 @@
 //                 row's top-k (k <= 16: a sorted list held in registers for
 //                 the whole item, each candidate placed in one step of
 //                 independent compares;
-//                 larger k: a heap in shared memory with the worst entry at
-//                 the root; 16, 32, 48 or 64 slots), publish the new
+//                 larger k: a four-ary heap in shared memory with the worst
+//                 entry at the root; 32, 48 or 64 slots), publish the new
 //                 threshold, which the filter reads every tile, and after an
 //                 item's last batch compute the softmax over the kept scores,
 //                 lse, and the weighted sum of the kept V rows (16-byte loads)
@@ -105,7 +105,10 @@ struct Cfg {
   static constexpr int kBoxBytes = kRegions * kRegionBytes;   // a 128-row box, all of d
   static constexpr int kQBytes = kMT * kBoxBytes;             // the item's Q tiles
   static constexpr int kStageBytes = kBoxBytes;               // one K tile (128 keys)
-  static constexpr int kListStride = KCAP + 1;                // list slots per row (+1: banks)
+  // list slots per row: KCAP + 1 for the register-list path (+1: banks); for
+  // the heap, 3 slots of lead so that each node's four children are one
+  // aligned 16-byte quad, rounded up to a multiple of 4 (16-byte rows)
+  static constexpr int kListStride = KCAP == kRegK ? KCAP + 1 : KCAP + 4;
   static constexpr int kListBytes = 2 * kListStride * kRows * 4;
   // One record buffer: per row r records of 16 scores (+4 floats: banks),
   // their first keys, and the row's record count.
@@ -178,11 +181,10 @@ __device__ __forceinline__ float max16(const float* x) {
 // first, kept in the insert thread's registers during an item and written
 // here for the softmax and gather: the first kRegK - k slots hold +inf
 // sentinels and the k real entries follow, so the k-th best is always the
-// last slot.  For larger KCAP the k
-// entries form a binary heap with the worst entry at the root (slot 0):
-// entry a is worse than entry b when a's score is smaller, or equal with a
-// larger key; the root's score is the row's threshold.  Unused entries hold
-// -inf and key -1.
+// last slot.  For larger KCAP the k entries, from slot 3 of the line on,
+// form a four-ary heap with the worst entry at the root: entry a is worse
+// than entry b when a's score is smaller, or equal with a larger key; the
+// root's score is the row's threshold.  Unused entries hold -inf and key -1.
 template <int KCAP>
 __device__ __forceinline__ int first_slot(int k) {
   return KCAP == kRegK ? kRegK - k : 0;
@@ -210,27 +212,25 @@ __device__ __forceinline__ bool worse(float sa, int ja, float sb, int jb) {
   return sa < sb || (sa == sb && ja > jb);
 }
 
-// Put (s, j) at slot `pos` of the heap of n entries and sift it down to
-// where both children are no worse than it.
-__device__ __forceinline__ void heap_sift(float* H, int* J, int n, int pos, float s, int j) {
+// Four-ary heap (children of p: 4p+1 .. 4p+4).  H + 1 and J + 1 are 16-byte
+// aligned, so each node's children are read as one float4 and one int4;
+// children at or past n count as +inf (never the worst).  Put (s, j) at
+// slot `pos` and sift it down to where all its children are no worse.
+__device__ __forceinline__ void heap4_sift(float* H, int* J, int n, int pos, float s, int j) {
   for (;;) {
-    const int l = 2 * pos + 1;
-    if (l >= n) break;
-    int c = l;
-    float cs = H[l];
-    int cj = J[l];
-    if (l + 1 < n) {
-      const float rs = H[l + 1];
-      const int rj = J[l + 1];
-      if (worse(rs, rj, cs, cj)) {
-        c = l + 1;
-        cs = rs;
-        cj = rj;
-      }
-    }
-    if (!worse(cs, cj, s, j)) break;
-    H[pos] = cs;
-    J[pos] = cj;
+    const int c0 = 4 * pos + 1;
+    if (c0 >= n) break;
+    const float4 cs = *reinterpret_cast<const float4*>(H + c0);
+    const int4 cj = *reinterpret_cast<const int4*>(J + c0);
+    int c = c0;
+    float ws = cs.x;
+    int wj = cj.x;
+    if (c0 + 1 < n && worse(cs.y, cj.y, ws, wj)) { c = c0 + 1; ws = cs.y; wj = cj.y; }
+    if (c0 + 2 < n && worse(cs.z, cj.z, ws, wj)) { c = c0 + 2; ws = cs.z; wj = cj.z; }
+    if (c0 + 3 < n && worse(cs.w, cj.w, ws, wj)) { c = c0 + 3; ws = cs.w; wj = cj.w; }
+    if (!worse(ws, wj, s, j)) break;
+    H[pos] = ws;
+    J[pos] = wj;
     pos = c;
   }
   H[pos] = s;
@@ -245,7 +245,7 @@ __device__ __forceinline__ void heap_to_sorted(float* H, int* J, int n) {
     const int j = J[end];
     H[end] = H[0];
     J[end] = J[0];
-    heap_sift(H, J, end, 0, s, j);
+    heap4_sift(H, J, end, 0, s, j);
   }
 }
 
@@ -334,8 +334,10 @@ __device__ __forceinline__ float insert_in_regs(float (&L)[kRegK], int (&J)[kReg
 }
 
 // Insertion for larger k: every recorded score that still beats the root of
-// the row's heap replaces the root and sifts down (log k steps in shared
-// memory, whatever the candidate's rank).  Returns the new threshold.
+// the row's heap replaces the root and sifts down (log4 k levels in shared
+// memory, one 16-byte load of scores and one of keys per level, whatever the
+// candidate's rank; a four-ary heap measured 1-5% faster for the whole
+// kernel than a binary one at k = 45 and 64).  Returns the new threshold.
 template <int NREC>
 __device__ __forceinline__ float insert_heap(float* H, int* J, const float* rs, const int* rj,
                                              int rn, float thr, int k) {
@@ -343,7 +345,7 @@ __device__ __forceinline__ float insert_heap(float* H, int* J, const float* rs, 
   float s;
   int jn;
   while (next_candidate(m, rs, rj, thr, s, jn)) {
-    heap_sift(H, J, k, 0, s, jn);
+    heap4_sift(H, J, k, 0, s, jn);
     thr = H[0];
   }
   __syncwarp();
@@ -715,7 +717,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           RJ[t] = -1;
         }
       } else {
-        list_reset<KCAP>(L, J, p.k);
+        list_reset<KCAP>(L + 3, J + 3, p.k);
       }
       float thr = -INFINITY;
       ++item_no;
@@ -733,7 +735,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if constexpr (KCAP == kRegK)
           thr = insert_in_regs<NR>(RL, RJ, rs, rj, rn, thr);
         else
-          thr = insert_heap<NR>(L, J, rs, rj, rn, thr, p.k);
+          thr = insert_heap<NR>(L + 3, J + 3, rs, rj, rn, thr, p.k);
         {
           // Publish the row's threshold with the item it belongs to, in one
           // 8-byte store, for the filter to raise its own.
@@ -755,9 +757,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
       if (tile_on && i < it.q1) {
-        if (KCAP != kRegK) heap_to_sorted(L, J, p.k);
-        const float* Lf = L + first_slot<KCAP>(p.k);
-        const int* Jf = J + first_slot<KCAP>(p.k);
+        if (KCAP != kRegK) heap_to_sorted(L + 3, J + 3, p.k);
+        const float* Lf = L + (KCAP == kRegK ? first_slot<KCAP>(p.k) : 3);
+        const int* Jf = J + (KCAP == kRegK ? first_slot<KCAP>(p.k) : 3);
         int cnt = 0;
         while (cnt < p.k && Jf[cnt] >= 0) ++cnt;
         // Softmax over the kept scaled scores, lse, weighted sum of V rows.
