@@ -281,6 +281,7 @@ class Case:
             self.dK = torch.empty_like(self.dQ)
             self.dV = torch.empty_like(self.dQ)
         self.flops = _score_flops(inp["offsets"], H, d)
+        self.scores = int(round(self.flops / (2 * d)))  # H * sum_g n_g^2 (query, key) pairs
         self.elem = self.g["Q"].element_size()
 
     def fwd(self, stream, k=None, idx=None):
@@ -324,6 +325,18 @@ def time_case(case, stream, steps, warmup, flush, clock=None, k=None, idx=None):
             bwd_ms.append(e1.elapsed_time(e2))
             mhz.append(clock.read() if clock else None)
     return fwd_ms, bwd_ms, mhz
+
+
+def _filter_roofline(scores: int, ms: float, sms: int, mhz) -> dict:
+    """The forward's second bound: its top-k filter reduces every score once
+    on the ALU pipe (a group's maximum of 16 scores is 15 two-input maxima,
+    or 8 three-input ones at half rate).  That pipe reduces 16 values per
+    clock per SM sub-partition, 64 per SM: 148 x 64 x clock scores/s."""
+    mhz = float(mhz or 1965.0)
+    peak = sms * 64 * mhz * 1e6
+    got = scores / (ms * 1e-3)
+    return {"bound": "alu", "scores": scores, "scores_per_s": got, "peak_scores_per_s": peak,
+            "frac": got / peak, "peak_from": f"{sms} SMs x 64 ALU lanes x {mhz:.0f} MHz"}
 
 
 def _fp32_fma_peak_tflops(sms: int, mhz: float) -> float:
@@ -573,7 +586,9 @@ def run_ours(args, ws, rank, local):
                          binding.kmip_fwd_path(d, k, binding.dtype_code(g["Q"].dtype)), "?")},
         "phases": {
             "fwd": {"ms": ms_fwd, "score_tflops": achieved, "frac_bf16_peak": achieved / peak,
-                    "gather_bytes_per_launch": N * H * _gather_bytes_per_unit(d, k, case.elem)},
+                    "gather_bytes_per_launch": N * H * _gather_bytes_per_unit(d, k, case.elem),
+                    "topk_filter": _filter_roofline(case.scores, ms_fwd, sms,
+                                                    clocks.get("sm_max_mhz"))},
             "gather_stage": {"kernel": "kmip_attn_gather (softmax + V gather over the forward's sets)",
                              "ms": gat_ms_mean, "algorithmic_bytes": gat_bytes,
                              "gbs": gat_bytes / (gat_ms_mean * 1e-3) / 1e9,
