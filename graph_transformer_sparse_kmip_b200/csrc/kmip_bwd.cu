@@ -8,6 +8,14 @@
 //   dS_j = p_j (dP_j - D),        dQ_i = scale sum_j dS_j K_j,
 //   dK_j += scale dS_j Q_i,       dV_j += p_j dO_i.
 //
+// p_j is taken as exp(scale s_j - lse) over the sum of those terms, the
+// softmax of the scores as this kernel recomputes them: lse (from the
+// forward) only shifts the exponent, and the forward's scores may differ from
+// these in the last bits (another summation order), which would leave the
+// p_j summing to 1 only up to rounding; when one key takes nearly all the
+// weight, dS_j = p_j (dP_j - D) cancels and that mismatch, not the
+// arithmetic of this kernel, would set its error.
+//
 // One warp per (query, head).  The d columns are split into 16-byte slices
 // (8 bf16 or 4 fp32 values per lane), so one warp instruction touches
 // 32 / (d / slice) kept rows at once with coalesced 16-byte loads.  Pass 1
@@ -59,7 +67,7 @@ bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restric
     const int32_t* ir = idx + pr * k;
 
     // Pass 1: p_j and dP_j of every kept key.
-    float Dsum = 0.f;
+    float Dsum = 0.f, Psum = 0.f;
     for (int ps = 0; ps < npass; ++ps) {
       const int t = ps * RPP + rs;
       int j = t < k ? ir[t] : -1;
@@ -96,9 +104,15 @@ bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restric
         }
       }
       Dsum = fmaf(p, dp, Dsum);  // identical in the LPR lanes of a row
+      Psum += p;
     }
 #pragma unroll
-    for (int o = LPR; o < 32; o <<= 1) Dsum += __shfl_xor_sync(0xffffffffu, Dsum, o);
+    for (int o = LPR; o < 32; o <<= 1) {
+      Dsum += __shfl_xor_sync(0xffffffffu, Dsum, o);
+      Psum += __shfl_xor_sync(0xffffffffu, Psum, o);
+    }
+    const float inv = Psum > 0.f ? 1.f / Psum : 0.f;
+    Dsum *= inv;
     __syncwarp();
 
     // Pass 2: dS_j, dQ accumulation, dK/dV scatter.
@@ -110,7 +124,7 @@ bwd_kernel(const T* __restrict__ dO, const T* __restrict__ Q, const T* __restric
       int j = t < k ? ir[t] : -1;
       if (j >= N || j < -1) j = -1;
       if (j >= 0) {
-        const float p = sp[warp][t];
+        const float p = sp[warp][t] * inv;
         const float ds = p * (sdp[warp][t] - Dsum);
         const int64_t kb = (int64_t)j * HD + (base % HD) + cs;
         float kv[VN];
