@@ -71,3 +71,39 @@ def test_random_shapes(dev, i):
                              dO=inp["dO"])
     for name, got in (("out", out), ("lse", lse), ("dQ", dQ), ("dK", dK), ("dV", dV)):
         check_values(name, got, given[name], dt)
+
+
+@pytest.mark.parametrize("i", range(0, N_CASES, 2))
+def test_random_shapes_other_entry_points(dev, i):
+    """The same seeded cases through the deterministic backward, the gather
+    stage, the all-key diagnostics and the no-allocation forward."""
+    sizes, H, d, k, dtype, scale = _case(i)
+    inp = wl.random_case(sizes, H=H, d=d, dtype=dtype, seed=7000 + i)
+    g = {n: t.to(dev) for n, t in inp.items()}
+    out, idx, lse = binding.attn_fwd(g["Q"], g["K"], g["V"], k, scale, g["offsets"])
+    det = binding.attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, scale, deterministic=True)
+    det2 = binding.attn_bwd(g["dO"], g["Q"], g["K"], g["V"], idx, lse, scale, deterministic=True)
+    o_g, l_g = binding.attn_gather(g["Q"], g["K"], g["V"], idx, scale)
+    o_d, i_d, l_d, lse_all = binding.attn_fwd_diag(g["Q"], g["K"], g["V"], k, scale, g["offsets"])
+    N = g["Q"].shape[0]
+    o_n, i_n, l_n = torch.empty_like(out), torch.empty_like(idx), torch.empty_like(lse)
+    rc = binding.kmip_attn_fwd_noalloc(g["Q"], g["K"], g["V"], g["offsets"], N, H, d, k, scale,
+                                       o_n, i_n, l_n)
+    assert rc == 0, binding.kmip_error_string(rc)
+    torch.cuda.synchronize()
+    binding.check_status()
+
+    for a, b in zip(det, det2):
+        assert torch.equal(a, b), "deterministic backward differs between two runs"
+    assert torch.equal(i_d, idx) and torch.equal(o_d, out) and torch.equal(l_d, lse)
+    assert torch.equal(i_n, idx) and torch.equal(o_n, out) and torch.equal(l_n, lse)
+
+    dt = inp["Q"].dtype
+    given = oracle.given_idx(inp["Q"], inp["K"], inp["V"], idx.cpu(), inp["offsets"], scale,
+                             dO=inp["dO"])
+    for name, got in zip(("dQ", "dK", "dV"), det):
+        check_values("deterministic " + name, got, given[name], dt)
+    check_values("gather out", o_g, given["out"], dt)
+    check_values("gather lse", l_g, given["lse"], dt)
+    full = oracle.full_attention(inp["Q"], inp["K"], inp["V"], inp["offsets"], scale)
+    check_values("lse_all", lse_all, full["lse"], dt)
