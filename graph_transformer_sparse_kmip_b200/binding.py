@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "KMIP_OK", 1: "KMIP_ERR_INVALID_ARG", 2: "KMIP_ERR_UNSUPPORTE
                 6: "KMIP_ERR_BAD_INDEX", 7: "KMIP_ERR_SCRATCH_LIMIT"}
 EXPORTED = ("kmip_attn_fwd", "kmip_attn_fwd_noalloc", "kmip_attn_fwd_diag", "kmip_attn_bwd",
             "kmip_attn_bwd_deterministic", "kmip_attn_gather", "kmip_get_status",
-            "kmip_scratch_usage", "kmip_error_string",
+            "kmip_scratch_usage", "kmip_scratch_trim", "kmip_error_string",
             "kmip_fwd_path", "kmip_version")
 
 _lib = None
@@ -65,6 +65,8 @@ def load() -> ctypes.CDLL:
     lib.kmip_get_status.restype = I32
     lib.kmip_scratch_usage.argtypes = [P, P, I32]
     lib.kmip_scratch_usage.restype = I32
+    lib.kmip_scratch_trim.argtypes = []
+    lib.kmip_scratch_trim.restype = I32
     lib.kmip_error_string.argtypes = [I32]
     lib.kmip_error_string.restype = ctypes.c_char_p
     lib.kmip_test_wait_timeout.argtypes = [P, I32]
@@ -230,6 +232,14 @@ def kmip_scratch_usage(reset_high: bool = False):
     if rc:
         raise KmipError(rc, "kmip_scratch_usage")
     return int(r.value), int(h.value)
+
+
+def kmip_scratch_trim():
+    """Return the library's unused pool memory on the current device (after
+    the streams that used the library have been synchronised)."""
+    rc = load().kmip_scratch_trim()
+    if rc:
+        raise KmipError(rc, "kmip_scratch_trim")
 
 
 def kmip_version() -> int:

@@ -127,6 +127,25 @@ cudaError_t scratch_usage(uint64_t* reserved, uint64_t* used_high, bool reset_hi
   return cudaSuccess;
 }
 
+// Trim the library's pool on the current device and reset what it keeps.
+cudaError_t scratch_trim() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaMemPool_t pool = g_pool[dev];
+  if (!pool) return cudaSuccess;
+  uint64_t zero = 0;
+  cudaError_t e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &zero);
+  if (e == cudaSuccess) e = cudaMemPoolTrimTo(pool, 0);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e;
+  }
+  g_pool_keep[dev] = 0;
+  return cudaSuccess;
+}
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
@@ -316,6 +335,10 @@ KMIP_EXPORT kmip_status_t kmip_scratch_usage(uint64_t* reserved, uint64_t* used_
                                              int reset_high) {
   return kmip::scratch_usage(reserved, used_high, reset_high != 0) == cudaSuccess ? KMIP_OK
                                                                                   : KMIP_ERR_CUDA;
+}
+
+KMIP_EXPORT kmip_status_t kmip_scratch_trim(void) {
+  return kmip::scratch_trim() == cudaSuccess ? KMIP_OK : KMIP_ERR_CUDA;
 }
 
 KMIP_EXPORT const char* kmip_error_string(kmip_status_t s) {

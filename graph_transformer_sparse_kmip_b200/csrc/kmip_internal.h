@@ -102,6 +102,7 @@ int device_sm_count();
 // current device (kmip_abi.cu); free with cudaFreeAsync on the same stream.
 cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream);
 cudaError_t scratch_usage(uint64_t* reserved, uint64_t* used_high, bool reset_high);
+cudaError_t scratch_trim();
 
 // Per-device status word address (nullptr if it cannot be resolved).
 int* status_ptr();

@@ -243,6 +243,16 @@ int kmip_fwd_path(int d, int k, kmip_dtype_t dtype);
  */
 kmip_status_t kmip_scratch_usage(uint64_t* reserved, uint64_t* used_high, int reset_high);
 
+/*
+ * Returns the memory the library's pool on the current device keeps but
+ * does not use to the device (cudaMemPoolTrimTo), and lets the pool keep
+ * nothing between calls until the next allocating call raises that again.
+ * Call it once the streams that ran library calls on the device have been
+ * synchronised: scratch still in use by queued work is not returned.
+ * Returns KMIP_OK (also when the pool does not exist yet) or KMIP_ERR_CUDA.
+ */
+kmip_status_t kmip_scratch_trim(void);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char* kmip_error_string(kmip_status_t status);
 

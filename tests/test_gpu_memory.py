@@ -58,3 +58,10 @@ def test_memory_is_linear_in_n():
     kept = N * H * w.k
     assert 20 * kept <= high2 <= 40 * kept + 8 * N * H + (4 << 20), (high2, kept)
     assert reserved2 >= high2
+
+    # trimming returns the kept memory once the work is done
+    torch.cuda.synchronize()
+    binding.kmip_scratch_trim()
+    reserved3, _ = binding.kmip_scratch_usage()
+    assert reserved3 < reserved2, (reserved3, reserved2)
+    assert reserved3 <= 64 << 20, reserved3
