@@ -150,7 +150,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -185,7 +185,7 @@ class ClockSampler:
         rows = self._rows()
         window = "timed region"
         if self.window and self.window[1]:
-            # a sample describes the 100 ms before it: keep those that end
+            # a sample describes the 50 ms before it: keep those that end
             # inside the window, and the first one after it
             a, b = self.window
             inside = [r for r in rows if a <= r[0] <= b]
